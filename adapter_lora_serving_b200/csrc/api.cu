@@ -1,0 +1,442 @@
+// C-ABI entry points: host-side validation, regime choice and launches.
+// Nothing here synchronises with the device or allocates memory.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/lora_delta.h"
+#include "kernels.h"
+#include "sgmv.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+lora_status fail(lora_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+lora_status ok() {
+  g_last_error[0] = '\0';
+  return LORA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+lora_status cuda_fail(cudaError_t err, const char* what, const char* why) {
+  if (why != nullptr) return fail(LORA_ERR_UNSUPPORTED, "%s: %s", what, why);
+  return fail(LORA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+// Checks shared by every linear / embedding entry point.  Fills slice_off.
+lora_status check_common(const char* op, int32_t T, int32_t in_features, int32_t slots,
+                         int32_t R, int32_t num_slices, const int32_t* out_slices,
+                         bool need_out, int* slice_off, int* out_total) {
+  if (T < 0) return fail(LORA_ERR_INVALID, "%s: T = %d < 0", op, T);
+  if (slots < 0) return fail(LORA_ERR_INVALID, "%s: slots = %d < 0", op, slots);
+  if (slots > LORA_MAX_SLOTS)
+    return fail(LORA_ERR_UNSUPPORTED, "%s: slots = %d > %d", op, slots, LORA_MAX_SLOTS);
+  if (R <= 0 || R % 8 != 0)
+    return fail(LORA_ERR_INVALID, "%s: R = %d must be a positive multiple of 8", op, R);
+  if (in_features <= 0 || in_features % 8 != 0)
+    return fail(LORA_ERR_INVALID, "%s: in_features = %d must be a positive multiple of 8", op,
+                in_features);
+  if (num_slices < 1 || num_slices > LORA_MAX_SLICES)
+    return fail(LORA_ERR_INVALID, "%s: num_slices = %d outside [1, %d]", op, num_slices,
+                LORA_MAX_SLICES);
+  slice_off[0] = 0;
+  if (need_out) {
+    if (out_slices == nullptr) return fail(LORA_ERR_INVALID, "%s: out_slices is NULL", op);
+    long long tot = 0;
+    for (int i = 0; i < num_slices; ++i) {
+      if (out_slices[i] <= 0 || out_slices[i] % 8 != 0)
+        return fail(LORA_ERR_INVALID, "%s: out_slices[%d] = %d must be a positive multiple of 8",
+                    op, i, out_slices[i]);
+      tot += out_slices[i];
+      if (tot > (1 << 30)) return fail(LORA_ERR_UNSUPPORTED, "%s: out too large", op);
+      slice_off[i + 1] = (int)tot;
+    }
+    *out_total = (int)tot;
+  } else {
+    for (int i = 0; i < num_slices; ++i) slice_off[i + 1] = 0;
+    *out_total = 0;
+  }
+  for (int i = num_slices + 1; i <= LORA_MAX_SLICES; ++i) slice_off[i] = slice_off[num_slices];
+  return LORA_OK;
+}
+
+lora_status check_ptrs(const char* op, std::initializer_list<std::pair<const void*, const char*>> p16,
+                       std::initializer_list<std::pair<const void*, const char*>> p4) {
+  for (auto& q : p16) {
+    if (q.first == nullptr) return fail(LORA_ERR_INVALID, "%s: %s is NULL", op, q.second);
+    if (!aligned16(q.first))
+      return fail(LORA_ERR_INVALID, "%s: %s is not 16-byte aligned", op, q.second);
+  }
+  for (auto& q : p4) {
+    if (q.first == nullptr) return fail(LORA_ERR_INVALID, "%s: %s is NULL", op, q.second);
+    if (!aligned4(q.first))
+      return fail(LORA_ERR_INVALID, "%s: %s is not 4-byte aligned", op, q.second);
+  }
+  return LORA_OK;
+}
+
+bool bgmv_fits(int S, int R) { return S * lora::round_up_i(R, 16) <= lora::kMaxSRp; }
+
+int resolve(int regime, int op, int T, int slots, int R, int S) {
+  if (regime == LORA_REGIME_BGMV || regime == LORA_REGIME_SGMV) return regime;
+  (void)op;
+  // Many tokens per slot on average: tensor-core tiles over slot segments.
+  if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024)
+    return LORA_REGIME_SGMV;
+  return LORA_REGIME_BGMV;
+}
+
+int linear_items_bound(int T, int slots, int tile) {
+  const long long b = (long long)slots + ((long long)T + tile - 1) / tile;
+  return (int)(b > (1LL << 30) ? (1LL << 30) : b);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lora_status_string(lora_status status) {
+  switch (status) {
+    case LORA_OK: return "LORA_OK";
+    case LORA_ERR_INVALID: return "LORA_ERR_INVALID";
+    case LORA_ERR_UNSUPPORTED: return "LORA_ERR_UNSUPPORTED";
+    case LORA_ERR_WORKSPACE: return "LORA_ERR_WORKSPACE";
+    case LORA_ERR_CUDA: return "LORA_ERR_CUDA";
+  }
+  return "LORA_ERR_UNKNOWN";
+}
+
+const char* lora_last_error(void) { return g_last_error; }
+
+const char* lora_version(void) { return "lora_delta 0.1.0 sm_100a"; }
+
+int32_t lora_resolve_regime(int32_t op, int32_t T, int32_t slots, int32_t R, int32_t num_slices) {
+  if (op == LORA_OP_EXPERT_APPLY) return LORA_REGIME_BGMV;
+  return resolve(LORA_REGIME_AUTO, op, T, slots, R, num_slices);
+}
+
+int32_t lora_plan_tile(int32_t op, int32_t regime) {
+  if (op == LORA_OP_EXPERT_APPLY) return lora::kTT;
+  if (regime == LORA_REGIME_SGMV) return lora::kSgmvTileM;
+  return lora::kTT;
+}
+
+size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R, int32_t num_slices,
+                            int32_t regime) {
+  if (op != LORA_OP_APPLY_LINEAR || T <= 0 || R <= 0 || num_slices <= 0) return 0;
+  const int reg = resolve(regime, op, T, slots, R, num_slices);
+  if (reg != LORA_REGIME_SGMV) return 0;
+  return lora::sgmv_workspace_bytes(T, R, num_slices);
+}
+
+lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* ranks,
+                        const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
+                        int32_t in_features, int32_t slots, int32_t R, int32_t num_slices,
+                        int32_t regime, uint32_t* err_flags, void* stream) {
+  const char* op = "lora_shrink";
+  lora::BgmvParams p = {};
+  int out = 0;
+  lora_status st = check_common(op, T, in_features, slots, R, num_slices, nullptr, false,
+                                p.slice_off, &out);
+  if (st != LORA_OK) return st;
+  if (T == 0 || slots == 0) return ok();
+  st = check_ptrs(op, {{x, "x"}, {h, "h"}, {a, "a"}},
+                  {{ranks, "ranks"}, {token_order, "token_order"}, {slot_indptr, "slot_indptr"}});
+  if (st != LORA_OK) return st;
+  if (err_flags != nullptr && !aligned4(err_flags))
+    return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  const int reg = resolve(regime, LORA_OP_SHRINK, T, slots, R, num_slices);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (reg == LORA_REGIME_SGMV) {
+    if (!lora::sgmv_supported(num_slices, R))
+      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+    const char* why = nullptr;
+    cudaError_t err = lora::sgmv_shrink_launch(x, a, h, ranks, token_order, slot_indptr, T,
+                                               in_features, slots, R, num_slices, err_flags, s,
+                                               &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
+  if (!bgmv_fits(num_slices, R))
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
+                num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  p.x = x; p.h = h; p.a = a; p.ranks = ranks; p.token_order = token_order;
+  p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T; p.in = in_features;
+  p.slots = slots; p.R = R; p.S = num_slices; p.out = 0;
+  const char* why = nullptr;
+  cudaError_t err = lora::bgmv_launch(lora::kModeShrink, p, linear_items_bound(T, slots, lora::kTT),
+                                      s, &why);
+  if (err != cudaSuccess) return cuda_fail(err, op, why);
+  return ok();
+}
+
+lora_status lora_expand(void* y, const float* h, const void* b, const int32_t* ranks,
+                        const float* scalings, const int32_t* token_order,
+                        const int32_t* slot_indptr, int32_t T, int32_t slots, int32_t R,
+                        const int32_t* out_slices, int32_t num_slices, int32_t regime,
+                        uint32_t* err_flags, void* stream) {
+  const char* op = "lora_expand";
+  lora::BgmvParams p = {};
+  int out = 0;
+  lora_status st =
+      check_common(op, T, 8, slots, R, num_slices, out_slices, true, p.slice_off, &out);
+  if (st != LORA_OK) return st;
+  if (T == 0 || slots == 0) return ok();
+  st = check_ptrs(op, {{y, "y"}, {h, "h"}, {b, "b"}},
+                  {{ranks, "ranks"}, {scalings, "scalings"}, {token_order, "token_order"},
+                   {slot_indptr, "slot_indptr"}});
+  if (st != LORA_OK) return st;
+  if (err_flags != nullptr && !aligned4(err_flags))
+    return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  const int reg = resolve(regime, LORA_OP_EXPAND, T, slots, R, num_slices);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (reg == LORA_REGIME_SGMV) {
+    if (!lora::sgmv_supported(num_slices, R))
+      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+    const char* why = nullptr;
+    cudaError_t err = lora::sgmv_expand_launch(y, h, nullptr, nullptr, b, ranks, scalings,
+                                               token_order, slot_indptr, T, 0, slots, R,
+                                               num_slices, p.slice_off, out, err_flags, s, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
+  if (!bgmv_fits(num_slices, R))
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
+                num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  p.y = y; p.h = const_cast<float*>(h); p.b = b; p.ranks = ranks; p.scalings = scalings;
+  p.token_order = token_order; p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T;
+  p.in = 8; p.slots = slots; p.R = R; p.S = num_slices; p.out = out;
+  const char* why = nullptr;
+  cudaError_t err = lora::bgmv_launch(lora::kModeExpand, p, linear_items_bound(T, slots, lora::kTT),
+                                      s, &why);
+  if (err != cudaSuccess) return cuda_fail(err, op, why);
+  return ok();
+}
+
+lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
+                              const int32_t* ranks, const float* scalings,
+                              const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
+                              int32_t in_features, int32_t slots, int32_t R,
+                              const int32_t* out_slices, int32_t num_slices, int32_t regime,
+                              void* workspace, size_t workspace_bytes, uint32_t* err_flags,
+                              void* stream) {
+  const char* op = "lora_apply_linear";
+  lora::BgmvParams p = {};
+  int out = 0;
+  lora_status st = check_common(op, T, in_features, slots, R, num_slices, out_slices, true,
+                                p.slice_off, &out);
+  if (st != LORA_OK) return st;
+  if (T == 0 || slots == 0) return ok();
+  st = check_ptrs(op, {{x, "x"}, {y, "y"}, {a, "a"}, {b, "b"}},
+                  {{ranks, "ranks"}, {scalings, "scalings"}, {token_order, "token_order"},
+                   {slot_indptr, "slot_indptr"}});
+  if (st != LORA_OK) return st;
+  if (err_flags != nullptr && !aligned4(err_flags))
+    return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, num_slices);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (reg == LORA_REGIME_SGMV) {
+    if (!lora::sgmv_supported(num_slices, R))
+      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+    const size_t need = lora::sgmv_workspace_bytes(T, R, num_slices);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(LORA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", op, need,
+                  workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned16(workspace))
+      return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
+    float* hws = static_cast<float*>(workspace);
+    const char* why = nullptr;
+    cudaError_t err = lora::sgmv_shrink_launch(x, a, hws, ranks, token_order, slot_indptr, T,
+                                               in_features, slots, R, num_slices, err_flags, s,
+                                               &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    err = lora::sgmv_expand_launch(y, hws, nullptr, nullptr, b, ranks, scalings, token_order,
+                                   slot_indptr, T, 0, slots, R, num_slices, p.slice_off, out,
+                                   nullptr, s, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
+  if (!bgmv_fits(num_slices, R))
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
+                num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  p.x = x; p.y = y; p.a = a; p.b = b; p.ranks = ranks; p.scalings = scalings;
+  p.token_order = token_order; p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T;
+  p.in = in_features; p.slots = slots; p.R = R; p.S = num_slices; p.out = out;
+  const char* why = nullptr;
+  cudaError_t err = lora::bgmv_launch(lora::kModeFused, p, linear_items_bound(T, slots, lora::kTT),
+                                      s, &why);
+  if (err != cudaSuccess) return cuda_fail(err, op, why);
+  return ok();
+}
+
+lora_status lora_gather_shrink(const int32_t* ids, float* h, const void* a, const int32_t* ranks,
+                               const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
+                               int32_t vocab, int32_t slots, int32_t R, int32_t num_slices,
+                               uint32_t* err_flags, void* stream) {
+  const char* op = "lora_gather_shrink";
+  lora::BgmvParams p = {};
+  int out = 0;
+  if (vocab <= 0) return fail(LORA_ERR_INVALID, "%s: vocab = %d must be positive", op, vocab);
+  lora_status st = check_common(op, T, 8, slots, R, num_slices, nullptr, false, p.slice_off, &out);
+  if (st != LORA_OK) return st;
+  if (T == 0 || slots == 0) return ok();
+  st = check_ptrs(op, {{h, "h"}, {a, "a"}},
+                  {{ids, "ids"}, {ranks, "ranks"}, {token_order, "token_order"},
+                   {slot_indptr, "slot_indptr"}});
+  if (st != LORA_OK) return st;
+  if (err_flags != nullptr && !aligned4(err_flags))
+    return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  if (!bgmv_fits(num_slices, R))
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
+                num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  p.ids = ids; p.h = h; p.a = a; p.ranks = ranks; p.token_order = token_order;
+  p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T; p.in = vocab; p.slots = slots;
+  p.R = R; p.S = num_slices; p.out = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const char* why = nullptr;
+  cudaError_t err = lora::bgmv_launch(lora::kModeGather, p, linear_items_bound(T, slots, lora::kTT),
+                                      s, &why);
+  if (err != cudaSuccess) return cuda_fail(err, op, why);
+  return ok();
+}
+
+lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, const void* b,
+                                 const int32_t* ranks, const float* scalings,
+                                 const int32_t* token_order, const int32_t* slot_indptr,
+                                 int32_t T, int32_t vocab, int32_t slots, int32_t R,
+                                 const int32_t* out_slices, int32_t num_slices, int32_t regime,
+                                 uint32_t* err_flags, void* stream) {
+  const char* op = "lora_apply_embedding";
+  lora::BgmvParams p = {};
+  int out = 0;
+  if (vocab <= 0) return fail(LORA_ERR_INVALID, "%s: vocab = %d must be positive", op, vocab);
+  lora_status st =
+      check_common(op, T, 8, slots, R, num_slices, out_slices, true, p.slice_off, &out);
+  if (st != LORA_OK) return st;
+  if (T == 0 || slots == 0) return ok();
+  st = check_ptrs(op, {{y, "y"}, {a, "a"}, {b, "b"}},
+                  {{ids, "ids"}, {ranks, "ranks"}, {scalings, "scalings"},
+                   {token_order, "token_order"}, {slot_indptr, "slot_indptr"}});
+  if (st != LORA_OK) return st;
+  if (err_flags != nullptr && !aligned4(err_flags))
+    return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  const int reg = resolve(regime, LORA_OP_APPLY_EMBEDDING, T, slots, R, num_slices);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (reg == LORA_REGIME_SGMV) {
+    if (!lora::sgmv_supported(num_slices, R))
+      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+    const char* why = nullptr;
+    cudaError_t err = lora::sgmv_expand_launch(y, nullptr, ids, a, b, ranks, scalings, token_order,
+                                               slot_indptr, T, vocab, slots, R, num_slices,
+                                               p.slice_off, out, err_flags, s, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
+  if (!bgmv_fits(num_slices, R))
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
+                num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  p.ids = ids; p.y = y; p.a = a; p.b = b; p.ranks = ranks; p.scalings = scalings;
+  p.token_order = token_order; p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T;
+  p.in = vocab; p.slots = slots; p.R = R; p.S = num_slices; p.out = out;
+  const char* why = nullptr;
+  cudaError_t err = lora::bgmv_launch(lora::kModeEmbed, p, linear_items_bound(T, slots, lora::kTT),
+                                      s, &why);
+  if (err != cudaSuccess) return cuda_fail(err, op, why);
+  return ok();
+}
+
+lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* a, const void* b,
+                              const int32_t* pair_index, const int32_t* ranks,
+                              const float* scalings, const int32_t* row_slot,
+                              const int32_t* expert_offsets, int32_t rows_cap, int32_t in_features,
+                              int32_t num_experts, int32_t slots, int32_t num_pairs, int32_t R,
+                              const int32_t* out_slices, int32_t num_slices, void* workspace,
+                              size_t workspace_bytes, uint32_t* err_flags, void* stream) {
+  const char* op = "lora_expert_apply";
+  (void)workspace;
+  (void)workspace_bytes;
+  lora::BgmvParams p = {};
+  int out = 0;
+  if (num_experts < 0 || num_experts > LORA_MAX_EXPERTS)
+    return fail(num_experts < 0 ? LORA_ERR_INVALID : LORA_ERR_UNSUPPORTED,
+                "%s: num_experts = %d outside [0, %d]", op, num_experts, LORA_MAX_EXPERTS);
+  if (num_pairs < 0) return fail(LORA_ERR_INVALID, "%s: num_pairs = %d < 0", op, num_pairs);
+  lora_status st = check_common(op, rows_cap, in_features, slots, R, num_slices, out_slices, true,
+                                p.slice_off, &out);
+  if (st != LORA_OK) return st;
+  if (rows_cap == 0 || slots == 0 || num_experts == 0 || num_pairs == 0) return ok();
+  st = check_ptrs(op, {{x_sorted, "x_sorted"}, {y_sorted, "y_sorted"}, {a, "a"}, {b, "b"}},
+                  {{pair_index, "pair_index"}, {ranks, "ranks"}, {scalings, "scalings"},
+                   {row_slot, "row_slot"}, {expert_offsets, "expert_offsets"}});
+  if (st != LORA_OK) return st;
+  if (err_flags != nullptr && !aligned4(err_flags))
+    return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  if (!bgmv_fits(num_slices, R))
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
+                num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  p.x = x_sorted; p.y = y_sorted; p.a = a; p.b = b; p.pair_index = pair_index; p.ranks = ranks;
+  p.scalings = scalings; p.row_slot = row_slot; p.expert_offsets = expert_offsets;
+  p.flags = err_flags; p.T = rows_cap; p.in = in_features; p.slots = slots; p.R = R;
+  p.S = num_slices; p.out = out; p.num_experts = num_experts; p.num_pairs = num_pairs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const char* why = nullptr;
+  const int bound = linear_items_bound(rows_cap, num_experts, lora::kTT);
+  cudaError_t err = lora::bgmv_launch(lora::kModeExpert, p, bound, s, &why);
+  if (err != cudaSuccess) return cuda_fail(err, op, why);
+  return ok();
+}
+
+lora_status lora_plan_linear(const int32_t* slot_indptr, const int32_t* ranks,
+                             const float* scalings, int32_t T, int32_t slots, int32_t R,
+                             int32_t tile, int32_t* plan_out, int32_t plan_cap,
+                             int32_t* plan_count, uint32_t* err_flags, void* stream) {
+  const char* op = "lora_plan_linear";
+  if (T < 0 || slots < 0 || R < 0 || tile <= 0 || plan_cap < 0)
+    return fail(LORA_ERR_INVALID, "%s: negative size or tile <= 0", op);
+  if (slots > LORA_MAX_SLOTS)
+    return fail(LORA_ERR_UNSUPPORTED, "%s: slots = %d > %d", op, slots, LORA_MAX_SLOTS);
+  lora_status st = check_ptrs(op, {}, {{slot_indptr, "slot_indptr"}, {ranks, "ranks"},
+                                       {plan_count, "plan_count"}});
+  if (st != LORA_OK) return st;
+  if (plan_cap > 0 && plan_out == nullptr) return fail(LORA_ERR_INVALID, "%s: plan_out is NULL", op);
+  cudaError_t err = lora::plan_linear_launch(slot_indptr, ranks, scalings, T, slots, R, tile,
+                                             plan_out, plan_cap, plan_count, err_flags,
+                                             reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, op, nullptr);
+  return ok();
+}
+
+lora_status lora_plan_expert(const int32_t* expert_offsets, const int32_t* pair_index,
+                             int32_t rows_cap, int32_t num_experts, int32_t slots,
+                             int32_t max_rows, int32_t* plan_out, int32_t plan_cap,
+                             int32_t* plan_count, uint32_t* err_flags, void* stream) {
+  const char* op = "lora_plan_expert";
+  if (rows_cap < 0 || num_experts < 0 || slots < 0 || max_rows <= 0 || plan_cap < 0)
+    return fail(LORA_ERR_INVALID, "%s: negative size or max_rows <= 0", op);
+  if (num_experts > LORA_MAX_EXPERTS)
+    return fail(LORA_ERR_UNSUPPORTED, "%s: num_experts = %d > %d", op, num_experts,
+                LORA_MAX_EXPERTS);
+  lora_status st = check_ptrs(op, {}, {{expert_offsets, "expert_offsets"},
+                                       {pair_index, "pair_index"}, {plan_count, "plan_count"}});
+  if (st != LORA_OK) return st;
+  if (plan_cap > 0 && plan_out == nullptr) return fail(LORA_ERR_INVALID, "%s: plan_out is NULL", op);
+  cudaError_t err = lora::plan_expert_launch(expert_offsets, pair_index, rows_cap, num_experts,
+                                             slots, max_rows, plan_out, plan_cap, plan_count,
+                                             err_flags, reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, op, nullptr);
+  return ok();
+}
+
+}  // extern "C"

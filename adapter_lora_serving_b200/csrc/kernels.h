@@ -1,0 +1,113 @@
+// Internal interface between the C-ABI entry points (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/lora_delta.h"
+
+namespace lora {
+
+// ---------------------------------------------------------------------------
+// BGMV regime: one thread-block cluster of kGroup CTAs per work item of at
+// most kTT tokens of one slot.  Each CTA reduces over 1/kGroup of the input
+// features (shrink), the cluster sums the partial h through distributed shared
+// memory, and each CTA then expands 1/kGroup of the output columns.
+// ---------------------------------------------------------------------------
+
+constexpr int kBgmvThreads = 256;
+constexpr int kTT = 16;          // tokens (sorted rows) per work item
+constexpr int kGroup = 8;        // CTAs per work item (cluster size)
+constexpr int kKB = 64;          // input features per pipeline stage
+constexpr int kNST = 4;          // pipeline stages
+constexpr int kRowStride = 144;  // bytes per staged row: 64 bf16 + 16 bytes of padding
+constexpr int kMaxCombosPerWarp = 4;  // (16-row tile, 8-token tile) pairs per warp
+constexpr int kMaxSRp = 256;     // num_slices * roundup(R, 16) limit of this regime
+
+enum BgmvMode : int {
+  kModeFused = 0,   // shrink + expand (apply_linear)
+  kModeShrink = 1,  // shrink only, h written to global
+  kModeExpand = 2,  // expand only, h read from global
+  kModeEmbed = 3,   // gather + expand (apply_embedding)
+  kModeGather = 4,  // gather only (gather_shrink)
+  kModeExpert = 5,  // MoE fold (shrink + expand per (expert chunk, slot))
+};
+
+struct BgmvParams {
+  const void* x;               // bf16 [rows, in]
+  void* y;                     // bf16 [rows, out]
+  const void* a;               // bf16 [W, S*R, in]
+  const void* b;               // bf16 [W, out, R]
+  float* h;                    // fp32 [T, S*R]
+  const int* ids;              // [T]
+  const int* ranks;            // [slots]
+  const float* scalings;       // [slots] (nullptr for unscaled operations)
+  const int* token_order;      // [T]
+  const int* slot_indptr;      // [slots+1]
+  const int* pair_index;       // [slots*E]
+  const int* row_slot;         // [rows_cap]
+  const int* expert_offsets;   // [E+1]
+  uint32_t* flags;
+  int T;          // tokens, or rows_cap for the expert fold
+  int in;         // input features (vocab for the embedding modes)
+  int slots;
+  int R;
+  int S;
+  int out;
+  int num_experts;
+  int num_pairs;
+  int slice_off[LORA_MAX_SLICES + 1];
+};
+
+struct BgmvLayout {
+  int prefix_off;
+  int misc_off;
+  int ring_off;
+  int hpart_off;
+  int hfull_off;
+  int total;
+  int srp;          // S * roundup(R, 16): h row stride in shared memory (floats)
+  int stage_bytes;  // bytes per pipeline stage
+};
+
+__host__ __device__ inline int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline int round_up_i(int a, int b) { return ceil_div_i(a, b) * b; }
+
+// Misc shared region (ints): tok[kTT], id[kTT], ctrl[8], scratch[8],
+// sub_s[kTT], sub_p[kTT], sub_cnt[kTT], sub_rows[kTT*kTT].
+constexpr int kMiscInts = kTT + kTT + 8 + 8 + 3 * kTT + kTT * kTT;
+
+__host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, int R) {
+  BgmvLayout L;
+  L.srp = S * round_up_i(R, 16);
+  L.stage_bytes = (L.srp + kTT) * kRowStride;
+  int off = 128;  // mbarriers
+  L.prefix_off = off;
+  off += round_up_i((npref + 1) * 4, 128);
+  L.misc_off = off;
+  off += round_up_i(kMiscInts * 4, 128);
+  L.ring_off = off;
+  const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpert);
+  if (ring) off += kNST * L.stage_bytes;
+  L.hpart_off = off;
+  if (ring) off += 2 * kTT * L.srp * 4;
+  L.hfull_off = off;
+  off += kTT * L.srp * 4;
+  L.total = off;
+  return L;
+}
+
+// Launchers (bgmv.cu).  Return a cudaError_t from the launch.
+cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,
+                        const char** why);
+
+// Device planners exposed for plan dumps (plan.cu).
+cudaError_t plan_linear_launch(const int* slot_indptr, const int* ranks, const float* scalings,
+                               int T, int slots, int R, int tile, int* plan_out, int plan_cap,
+                               int* plan_count, uint32_t* flags, cudaStream_t stream);
+cudaError_t plan_expert_launch(const int* offsets, const int* pair_index, int rows_cap, int E,
+                               int slots, int max_rows, int* plan_out, int plan_cap,
+                               int* plan_count, uint32_t* flags, cudaStream_t stream);
+
+}  // namespace lora

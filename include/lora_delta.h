@@ -1,0 +1,240 @@
+/*
+ * lora_delta.h -- C ABI of the B200 (sm_100a) batched multi-LoRA delta library.
+ *
+ * Each token (or sorted MoE row) carries an adapter slot.  The library adds
+ * the slot's low-rank delta to a projection's output in place:
+ *
+ *   shrink  h[t, i*R + r] = sum_k x[t, k] * a[slot, i*R + r, k]      (r < rank)
+ *   expand  y[t, off_i + j] += scaling[slot] * sum_{r<rank} h[t, i*R + r] * b[slot, off_i + j, r]
+ *
+ * Sources (page title, section):
+ *   mstar.engine.resources.lora.backend -- module text (shapes, slices),
+ *     LoraBackend.shrink / expand_fused / apply_linear_ / apply_ / gather_shrink,
+ *     and the addressing (token_order, slot_indptr) of shrink_reference,
+ *     expand_reference_ and gather_shrink_reference.
+ *   mstar.model.components.linear -- FusedColumnLinear (shards laid out in order).
+ *   spark_model/lora/expert_apply.rs -- expert_delta_workitems, fold_chunked,
+ *     apply_expert_lora_sorted (the expert fold over expert_offsets).
+ *   spark_model/lora/target.rs -- ExpertLoraLayer (sparse per-expert pairs,
+ *     adapted_experts), expert_router_bytes (uint4-aligned packed rank stride).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless marked "host".  bf16 tensors are
+ *     passed as void* and are row-major and contiguous.  Every device pointer
+ *     must be 16-byte aligned.
+ *   - The caller owns every buffer.  The library never allocates device
+ *     memory and keeps no state between calls except a per-device cache of
+ *     kernel attributes (SM count, occupancy).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronises with the host.  The launch shape
+ *     depends only on the scalar arguments, so calls can be captured in a CUDA
+ *     graph.
+ *   - Host-checkable errors return a non-LORA_OK status before anything is
+ *     launched.  lora_last_error() then gives a message (thread-local).
+ *   - Bad addressing that is only visible on the device is skipped, never
+ *     trapped, and ORed into *err_flags when err_flags is not NULL (bits
+ *     LORA_FLAG_*).  err_flags is never cleared by the library.
+ *   - Shape rules (uint4 = 16-byte packing of bf16 rows, after the packed rank
+ *     stride of expert_router_bytes): in_features % 8 == 0, R % 8 == 0,
+ *     every out_slices[i] % 8 == 0, 1 <= num_slices <= LORA_MAX_SLICES.
+ *
+ * Addressing (CSR by slot): slot s owns slot-sorted positions
+ * [slot_indptr[s], slot_indptr[s+1]); token_order[p] is the token at position p.
+ * A segment is used only if 0 <= lo <= hi <= T (else LORA_FLAG_BAD_INDPTR) and
+ * the slot's rank is in [0, R] (else LORA_FLAG_BAD_RANK).  Positions whose
+ * token is outside [0, T) are skipped (LORA_FLAG_BAD_TOKEN).  Tokens listed in
+ * no segment are untouched.  A slot with rank 0 -- or, for the operations
+ * that scale, scaling 0 -- leaves y bit-identical.  A token listed twice gives
+ * an unspecified result.
+ */
+#ifndef LORA_DELTA_H
+#define LORA_DELTA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LORA_API __attribute__((visibility("default")))
+#else
+#define LORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LORA_OK = 0,
+  LORA_ERR_INVALID = 1,      /* a host-checkable argument is wrong; nothing launched */
+  LORA_ERR_UNSUPPORTED = 2,  /* valid, but beyond this library's limits */
+  LORA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+  LORA_ERR_CUDA = 4          /* a CUDA runtime call or a launch failed */
+} lora_status;
+
+/* Device-side error flags, ORed into *err_flags. */
+#define LORA_FLAG_BAD_INDPTR  1u   /* a slot segment outside 0 <= lo <= hi <= T */
+#define LORA_FLAG_BAD_TOKEN   2u   /* token_order entry outside [0, T) */
+#define LORA_FLAG_BAD_RANK    4u   /* rank outside [0, R] */
+#define LORA_FLAG_BAD_SLOT    8u   /* MoE row_slot outside [-1, slots) */
+#define LORA_FLAG_BAD_PAIR   16u   /* MoE pair_index outside [-1, num_pairs) */
+#define LORA_FLAG_BAD_OFFSETS 32u  /* MoE expert offsets with start < 0, end > rows_cap or end < start */
+#define LORA_FLAG_TIMEOUT    64u   /* a bounded device wait expired; the call's output is incomplete */
+
+/* Regime hint.  AUTO picks from the scalar shapes only (tokens per slot). */
+#define LORA_REGIME_AUTO 0
+#define LORA_REGIME_BGMV 1   /* few tokens per slot: thread-block-cluster kernel, h kept on chip */
+#define LORA_REGIME_SGMV 2   /* many tokens per slot: tcgen05/TMEM tiles over slot segments */
+
+#define LORA_MAX_SLICES 8
+#define LORA_MAX_SLOTS 4096
+#define LORA_MAX_EXPERTS 4096
+
+/* Operation ids for lora_plan_tile / lora_workspace_bytes. */
+#define LORA_OP_SHRINK 0
+#define LORA_OP_EXPAND 1
+#define LORA_OP_APPLY_LINEAR 2
+#define LORA_OP_GATHER_SHRINK 3
+#define LORA_OP_APPLY_EMBEDDING 4
+#define LORA_OP_EXPERT_APPLY 5
+
+/*
+ * lora_shrink -- LoraBackend.shrink (mstar.engine.resources.lora.backend):
+ *   h[t] = x[t] @ a[slot(t)]^T over num_slices*R columns.
+ * x [T, in_features] bf16; a [slots, num_slices*R, in_features] bf16;
+ * h [T, num_slices*R] fp32 (written).  Only h[t, i*R + r] with r < rank of a
+ * live token's slot is written; every other entry is left as it was (the page
+ * allows anything there: the expand never reads it).
+ */
+LORA_API lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* ranks,
+                        const int32_t* token_order, const int32_t* slot_indptr,
+                        int32_t T, int32_t in_features, int32_t slots, int32_t R,
+                        int32_t num_slices, int32_t regime, uint32_t* err_flags,
+                        void* stream);
+
+/*
+ * lora_expand -- LoraBackend.expand_fused:
+ *   y[t, slice i] += scalings[slot(t)] * h[t, slice i cols < rank] @ b[slot(t), slice i]^T
+ * h [T, num_slices*R] fp32; b [slots, out, R] bf16 with out = sum(out_slices);
+ * y [T, out] bf16, in place: y = bf16_rne(float(y) + scaling * acc), acc in fp32.
+ * out_slices (host, num_slices entries): widths of the fused projection's
+ * outputs in column order (e.g. q, k, v).
+ */
+LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const int32_t* ranks,
+                        const float* scalings, const int32_t* token_order,
+                        const int32_t* slot_indptr, int32_t T, int32_t slots, int32_t R,
+                        const int32_t* out_slices, int32_t num_slices, int32_t regime,
+                        uint32_t* err_flags, void* stream);
+
+/*
+ * lora_apply_linear -- LoraBackend.apply_linear_ (shrink then expand, fused):
+ * same arguments as lora_shrink + lora_expand, with h kept on chip (BGMV) or in
+ * `workspace` (SGMV).  workspace must hold lora_workspace_bytes(
+ * LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, regime) bytes (may be NULL
+ * when that is 0).
+ */
+LORA_API lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
+                              const int32_t* ranks, const float* scalings,
+                              const int32_t* token_order, const int32_t* slot_indptr,
+                              int32_t T, int32_t in_features, int32_t slots, int32_t R,
+                              const int32_t* out_slices, int32_t num_slices, int32_t regime,
+                              void* workspace, size_t workspace_bytes, uint32_t* err_flags,
+                              void* stream);
+
+/*
+ * lora_gather_shrink -- LoraBackend.gather_shrink:
+ *   h[t, i*R + r] = a[slot(t), i*R + r, ids[t]]  (r < rank)
+ * ids [T] int32 token ids; a [slots, num_slices*R, vocab] bf16; h [T, num_slices*R]
+ * fp32.  An id outside [0, vocab) (e.g. -1 for an image position) contributes
+ * nothing: its h row is written as zeros.
+ */
+LORA_API lora_status lora_gather_shrink(const int32_t* ids, float* h, const void* a,
+                               const int32_t* ranks, const int32_t* token_order,
+                               const int32_t* slot_indptr, int32_t T, int32_t vocab,
+                               int32_t slots, int32_t R, int32_t num_slices,
+                               uint32_t* err_flags, void* stream);
+
+/*
+ * lora_apply_embedding -- LoraBackend.apply_ with embedding=True (gather, then
+ * expand; fused, h kept on chip).  A token whose id is outside [0, vocab)
+ * contributes nothing and its row of y stays bit-identical.
+ */
+LORA_API lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, const void* b,
+                                 const int32_t* ranks, const float* scalings,
+                                 const int32_t* token_order, const int32_t* slot_indptr,
+                                 int32_t T, int32_t vocab, int32_t slots, int32_t R,
+                                 const int32_t* out_slices, int32_t num_slices,
+                                 int32_t regime, uint32_t* err_flags, void* stream);
+
+/*
+ * lora_expert_apply -- the MoE expert fold (spark_model/lora/expert_apply.rs,
+ * apply_expert_lora_sorted, with the per-request slot routing the page plans
+ * for its grouped (slot, expert) kernel):
+ *   for every adapted expert e (ascending) with rows [expert_offsets[e],
+ *   expert_offsets[e+1]), for every row rho there whose slot s = row_slot[rho]
+ *   is >= 0 and whose pair p = pair_index[s*num_experts + e] is >= 0:
+ *     y_sorted[rho, slice i] += scalings[s] * (x_sorted[rho] @ a[p, slice i rows < rank]^T) @ b[p, slice i]^T
+ * The fold runs after the base grouped GEMM and before unpermute: for gate/up
+ * call it on the gate/up output (before silu_mul), for down on the down output.
+ * x_sorted [rows_cap, in_features] bf16; y_sorted [rows_cap, out] bf16 in place;
+ * a [num_pairs, num_slices*R, in_features]; b [num_pairs, out, R];
+ * pair_index [slots*num_experts] (-1 = not adapted); ranks, scalings [slots];
+ * row_slot [rows_cap] (-1 = no adapter); expert_offsets [num_experts+1].
+ * Planning happens on the device (no copy of expert_offsets to the host).
+ * workspace may be NULL when lora_workspace_bytes(LORA_OP_EXPERT_APPLY, ...) is 0.
+ */
+LORA_API lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* a,
+                              const void* b, const int32_t* pair_index, const int32_t* ranks,
+                              const float* scalings, const int32_t* row_slot,
+                              const int32_t* expert_offsets, int32_t rows_cap,
+                              int32_t in_features, int32_t num_experts, int32_t slots,
+                              int32_t num_pairs, int32_t R, const int32_t* out_slices,
+                              int32_t num_slices, void* workspace, size_t workspace_bytes,
+                              uint32_t* err_flags, void* stream);
+
+/*
+ * Workspace bytes an operation needs for these shapes and regime (0 if none).
+ * For LORA_OP_EXPERT_APPLY pass rows_cap as T and num_experts as slots.
+ */
+LORA_API size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R,
+                            int32_t num_slices, int32_t regime);
+
+/* The regime LORA_REGIME_AUTO resolves to for these scalar shapes. */
+LORA_API int32_t lora_resolve_regime(int32_t op, int32_t T, int32_t slots, int32_t R,
+                            int32_t num_slices);
+
+/* Positions (or sorted rows) per work item of an operation's kernel in a regime. */
+LORA_API int32_t lora_plan_tile(int32_t op, int32_t regime);
+
+/*
+ * lora_plan_linear -- runs the device work-item planner the kernels use and
+ * writes its plan: plan_out[3*i .. 3*i+2] = (slot, first position, count) for
+ * i < min(*plan_count, plan_cap); *plan_count (device int32) = number of items.
+ * scalings may be NULL (the unscaled operations: shrink, gather).  Slots are in
+ * ascending order, each cut into consecutive tiles of `tile` positions.
+ */
+LORA_API lora_status lora_plan_linear(const int32_t* slot_indptr, const int32_t* ranks,
+                             const float* scalings, int32_t T, int32_t slots, int32_t R,
+                             int32_t tile, int32_t* plan_out, int32_t plan_cap,
+                             int32_t* plan_count, uint32_t* err_flags, void* stream);
+
+/*
+ * lora_plan_expert -- the device expert planner (expert_delta_workitems then
+ * fold_chunked): plan_out[3*i..] = (expert, row_off, rows) per chunk of at most
+ * `max_rows` rows, experts ascending over the adapted set (experts holding a
+ * pair for any slot); *plan_count = number of chunks.
+ */
+LORA_API lora_status lora_plan_expert(const int32_t* expert_offsets, const int32_t* pair_index,
+                             int32_t rows_cap, int32_t num_experts, int32_t slots,
+                             int32_t max_rows, int32_t* plan_out, int32_t plan_cap,
+                             int32_t* plan_count, uint32_t* err_flags, void* stream);
+
+LORA_API const char* lora_status_string(lora_status status);
+LORA_API const char* lora_last_error(void);
+/* Library version, e.g. "lora_delta 0.1.0 sm_100a". */
+LORA_API const char* lora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_DELTA_H */

@@ -1,0 +1,118 @@
+"""The C-ABI library on a host without a GPU: it loads, exports every symbol the
+header declares, and rejects host-checkable mistakes before any CUDA call."""
+import os
+import re
+
+import pytest
+
+from adapter_lora_serving_b200 import lora as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_delta.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(L.LIB_PATH):
+        from adapter_lora_serving_b200 import build
+        build.build()
+    return L.load()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(lora_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_symbols_exported(lib):
+    declared = _declared()
+    assert "lora_apply_linear" in declared and "lora_expert_apply" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(L.EXPORTED) == declared
+
+
+def test_version(lib):
+    assert "sm_100a" in L.lora_version()
+
+
+FAKE = 1 << 20          # a 16-byte aligned, never dereferenced address
+
+
+def _apply(lib, **kw):
+    args = dict(x=FAKE, y=FAKE, a=FAKE, b=FAKE, ranks=FAKE, scalings=FAKE, token_order=FAKE,
+                slot_indptr=FAKE, T=16, in_features=64, slots=2, R=16, out_slices=(32,),
+                regime=L.LORA_REGIME_BGMV, ws=None, ws_bytes=0, flags=None)
+    args.update(kw)
+    sl = L._slices(args["out_slices"])
+    return lib.lora_apply_linear(args["x"], args["y"], args["a"], args["b"], args["ranks"],
+                                 args["scalings"], args["token_order"], args["slot_indptr"],
+                                 args["T"], args["in_features"], args["slots"], args["R"], sl,
+                                 len(args["out_slices"]), args["regime"], args["ws"],
+                                 args["ws_bytes"], args["flags"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(R=12),                       # not a multiple of 8
+    dict(R=0),
+    dict(in_features=60),
+    dict(out_slices=(20,)),
+    dict(out_slices=()),
+    dict(out_slices=(8,) * 9),        # more than LORA_MAX_SLICES
+    dict(T=-1),
+    dict(slots=-2),
+    dict(x=None),
+    dict(x=FAKE + 8),                 # not 16-byte aligned
+    dict(ranks=FAKE + 2),             # not 4-byte aligned
+    dict(flags=FAKE + 1),
+])
+def test_apply_linear_rejects(lib, kw):
+    assert _apply(lib, **kw) == L.LORA_ERR_INVALID
+    assert lib.lora_last_error().decode().startswith("lora_apply_linear")
+
+
+def test_limits_unsupported(lib):
+    assert _apply(lib, slots=5000) == L.LORA_ERR_UNSUPPORTED
+    # 3 slices of R=128 exceed the BGMV shared-memory tile
+    assert _apply(lib, R=128, out_slices=(8, 8, 8)) == L.LORA_ERR_UNSUPPORTED
+
+
+def test_empty_calls_launch_nothing(lib):
+    assert _apply(lib, T=0) == L.LORA_OK
+    assert _apply(lib, slots=0) == L.LORA_OK
+
+
+def test_other_entry_points_validate(lib):
+    sl = L._slices((16,))
+    assert lib.lora_expand(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 2, 10, sl, 1, 0, None,
+                           None) == L.LORA_ERR_INVALID
+    assert lib.lora_shrink(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 12, 2, 8, 1, 0, None,
+                           None) == L.LORA_ERR_INVALID
+    assert lib.lora_gather_shrink(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 0, 2, 8, 1, None,
+                                  None) == L.LORA_ERR_INVALID
+    assert lib.lora_apply_embedding(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, -5, 2, 8,
+                                    sl, 1, 0, None, None) == L.LORA_ERR_INVALID
+    assert lib.lora_expert_apply(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 64,
+                                 -1, 2, 4, 8, sl, 1, None, 0, None, None) == L.LORA_ERR_INVALID
+    assert lib.lora_expert_apply(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 64,
+                                 5000, 2, 4, 8, sl, 1, None, 0, None,
+                                 None) == L.LORA_ERR_UNSUPPORTED
+    assert lib.lora_plan_linear(FAKE, FAKE, None, 8, 2, 8, 0, FAKE, 4, FAKE, None,
+                                None) == L.LORA_ERR_INVALID
+    assert lib.lora_plan_expert(FAKE, FAKE, 8, 2, 2, 0, FAKE, 4, FAKE, None,
+                                None) == L.LORA_ERR_INVALID
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "LORA_OK"), (1, "LORA_ERR_INVALID"), (2, "LORA_ERR_UNSUPPORTED"),
+                       (3, "LORA_ERR_WORKSPACE"), (4, "LORA_ERR_CUDA")]:
+        assert lib.lora_status_string(code).decode() == name
+
+
+def test_host_queries(lib):
+    assert L.lora_plan_tile(L.LORA_OP_APPLY_LINEAR, L.LORA_REGIME_BGMV) == 16
+    assert L.lora_plan_tile(L.LORA_OP_EXPERT_APPLY, L.LORA_REGIME_AUTO) == 16
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
+                                  L.LORA_REGIME_BGMV) == 0
+    assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == L.LORA_REGIME_BGMV
