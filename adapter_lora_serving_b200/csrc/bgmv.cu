@@ -541,7 +541,9 @@ cudaError_t launch_mode(const BgmvParams& p, int max_items, cudaStream_t stream,
       *why = "shared memory needed by the BGMV kernel exceeds the device limit";
       return cudaErrorInvalidConfiguration;
     }
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+    // Allow the device maximum once: a later call with a smaller layout must
+    // not lower the limit a cached larger layout relies on.
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin);
     if (err != cudaSuccess) return err;
     int sms = 0;
     err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
