@@ -3,8 +3,8 @@
 // expert chunk and slot).
 //
 // Shrink: each CTA of the cluster owns 1/kGroup of the input features.  The
-// slot's live A rows and the item's x rows stream through a kNST-stage ring
-// of shared memory by bulk copies (the TMA engine) and feed m16n8k16 warp MMAs
+// slot's live A rows and the item's x rows are staged in shared memory by
+// coalesced 16-byte asynchronous copies and feed m16n8k16 warp MMAs
 // (fp32 accumulate).  The kGroup partial h tiles are summed in a fixed order
 // through distributed shared memory, so every CTA holds the same full h and
 // h never leaves the chip.
@@ -26,24 +26,23 @@ namespace lora {
 namespace {
 
 struct Smem {
-  uint64_t* bars;
   int* prefix;
   int* tok;
   int* ids;
-  int* ctrl;     // [0..1] item count, [2..3] sub-batch count (by parity), [4] abort
+  int* ctrl;     // [0] item count, [2..3] sub-batch count (by parity)
   int* scratch;
   int* sub_s;
   int* sub_p;
   int* sub_cnt;
   int* sub_rows;
   uint8_t* ring;
-  float* hpart;  // 2 buffers of kTT * srp
-  float* hfull;  // kTT * srp
+  float* hpart;     // 2 buffers of kTT * srp (cluster partial sums)
+  uint16_t* hhi;    // [S][kTT][hst]
+  uint16_t* hlo;    // [S][kTT][hst]
 };
 
 LORA_DEV Smem carve(uint8_t* base, const BgmvLayout& L) {
   Smem s;
-  s.bars = reinterpret_cast<uint64_t*>(base);
   s.prefix = reinterpret_cast<int*>(base + L.prefix_off);
   int* m = reinterpret_cast<int*>(base + L.misc_off);
   s.tok = m;
@@ -56,32 +55,73 @@ LORA_DEV Smem carve(uint8_t* base, const BgmvLayout& L) {
   s.sub_rows = s.sub_cnt + kTT;
   s.ring = base + L.ring_off;
   s.hpart = reinterpret_cast<float*>(base + L.hpart_off);
-  s.hfull = reinterpret_cast<float*>(base + L.hfull_off);
+  s.hhi = reinterpret_cast<uint16_t*>(base + L.hhi_off);
+  s.hlo = reinterpret_cast<uint16_t*>(base + L.hlo_off);
   return s;
 }
 
-// Shrink of one item over this CTA's share of the input features into
-// hpart[t * srp + i*Rpad + r] (t < kTT, every 16-row tile that holds a live
-// row).  kbc counts ring stages consumed so far (same in every thread).
+// Geometry of the shrink of one item on this CTA.
+struct ShrinkGeom {
+  int k0, k1, nkb;   // this CTA's input features [k0, k1), in stages of p.kb
+  int nrows_a;       // live A rows: S * rank
+};
+
+LORA_DEV ShrinkGeom shrink_geom(const BgmvParams& p, int rank, uint32_t crank) {
+  ShrinkGeom G;
+  const int kchunk = bgmv_kchunk(p.in);
+  G.k0 = min(p.in, (int)crank * kchunk);
+  G.k1 = min(p.in, G.k0 + kchunk);
+  G.nkb = ceil_div_i(G.k1 - G.k0, p.kb);
+  G.nrows_a = p.S * rank;
+  return G;
+}
+
+// Issue 16-byte copies of staged rows [row_lo, row_hi) of stage kb into ring
+// slot st.  Rows below nrows_a are live A rows; the next kTT rows are the
+// item's x rows (rows of invalid tokens are skipped).  A warp copies a row.
+LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                         const ShrinkGeom& G, int w, int rank, int kb, int st, int row_lo,
+                         int row_hi) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int kbase = G.k0 + kb * p.kb;
+  const int cpr = min(p.kb, G.k1 - kbase) >> 3;   // 16-byte chunks per row
+  const int Rpad = round_up_i(p.R, 16);
+  const uint32_t stage = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
+  for (int row = row_lo + warp; row < row_hi; row += kBgmvThreads / 32) {
+    const __nv_bfloat16* src;
+    uint32_t dst;
+    if (row < G.nrows_a) {
+      const int i = row / rank;
+      const int r = row - i * rank;
+      src = reinterpret_cast<const __nv_bfloat16*>(p.a) +
+            ((size_t)w * p.S * p.R + i * p.R + r) * p.in + kbase;
+      dst = stage + (uint32_t)((i * Rpad + r) * L.row_stride);
+    } else {
+      const int t = row - G.nrows_a;
+      const int tk = sm.tok[t];
+      if (tk < 0) continue;
+      src = reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)tk * p.in + kbase;
+      dst = stage + (uint32_t)((L.srp + t) * L.row_stride);
+    }
+    for (int c = lane; c < cpr; c += 32) cp_async16(dst + c * 16, src + c * 8);
+  }
+}
+
+// MMAs of the shrink over this CTA's input features into hpart[t * srp +
+// i*Rpad + r] (every 16-row tile holding a live row, t < 8*ceil(n/8)).  The
+// caller has issued the A rows of stage 0 (uncommitted); this issues the rest.
 LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                             uint32_t& kbc, int w, int rank, int n, int nvalid, uint32_t crank,
-                             float* hpart) {
+                             const ShrinkGeom& G, int w, int rank, int n, float* hpart) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int Rpad = round_up_i(p.R, 16);
-  const int kchunk = round_up_i(ceil_div_i(p.in, kGroup), kKB);
-  const int k0 = min(p.in, (int)crank * kchunk);
-  const int k1 = min(p.in, k0 + kchunk);
-  const int nkb = ceil_div_i(k1 - k0, kKB);
   const int tps = ceil_div_i(rank, 16);
   const int RT = p.S * tps;
   const int NTt = ceil_div_i(n, 8);
   const int combos = RT * NTt;
-  const int nrows_a = p.S * rank;
-  const __nv_bfloat16* abase =
-      reinterpret_cast<const __nv_bfloat16*>(p.a) + (size_t)w * p.S * p.R * p.in;
-  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(p.x);
+  const int stride = L.row_stride;
 
   float acc[kMaxCombosPerWarp][4];
 #pragma unroll
@@ -89,80 +129,53 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[c][q] = 0.f;
 
-  auto issue = [&](int kb, int st) {  // warp 0, converged
-    const int kbase = k0 + kb * kKB;
-    const int kv = min(kKB, k1 - kbase);
-    const uint32_t rowbytes = (uint32_t)kv * 2u;
-    uint8_t* stage = sm.ring + (size_t)st * L.stage_bytes;
-    if (lane == 0) mbar_arrive_expect_tx(&sm.bars[st], (uint32_t)(nrows_a + nvalid) * rowbytes);
-    __syncwarp();
-    for (int q = lane; q < nrows_a + n; q += 32) {
-      if (q < nrows_a) {
-        const int i = q / rank;
-        const int r = q - i * rank;
-        bulk_g2s(stage + (size_t)(i * Rpad + r) * kRowStride,
-                 abase + (size_t)(i * p.R + r) * p.in + kbase, rowbytes, &sm.bars[st]);
-      } else {
-        const int t = q - nrows_a;
-        const int tk = sm.tok[t];
-        if (tk >= 0)
-          bulk_g2s(stage + (size_t)(L.srp + t) * kRowStride, xb + (size_t)tk * p.in + kbase,
-                   rowbytes, &sm.bars[st]);
-      }
+  if (G.nkb > 0) {
+    issue_rows(p, L, sm, G, w, rank, 0, 0, G.nrows_a, G.nrows_a + n);
+    cp_async_commit();
+    if (G.nkb > 1 && p.nst == 2) {
+      issue_rows(p, L, sm, G, w, rank, 1, 1, 0, G.nrows_a + n);
+      cp_async_commit();
     }
-  };
-
-  volatile int* abort_flag = &sm.ctrl[4];
-  if (warp == 0 && *abort_flag == 0) {
-    for (int kb = 0; kb < min(nkb, kNST); ++kb) issue(kb, (int)((kbc + kb) % kNST));
   }
-  for (int kb = 0; kb < nkb; ++kb) {
-    const uint32_t g = kbc + kb;
-    const int st = (int)(g % kNST);
-    const uint32_t parity = (g / kNST) & 1u;
-    bool ok = (*abort_flag == 0);
-    if (ok && !mbar_wait(&sm.bars[st], parity)) {
-      ok = false;
-      *abort_flag = 1;
-      raise_flag(p.flags, LORA_FLAG_TIMEOUT);
-    }
-    if (ok) {
-      const int kv = min(kKB, k1 - (k0 + kb * kKB));
-      const int nks = ceil_div_i(kv, 16);
-      const uint32_t stage_addr = smem_u32(sm.ring + (size_t)st * L.stage_bytes);
+  for (int kb = 0; kb < G.nkb; ++kb) {
+    const int st = kb % p.nst;
+    if (kb + 1 < G.nkb && p.nst == 2) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncthreads();
+    const int kv = min(p.kb, G.k1 - (G.k0 + kb * p.kb));
+    const int nks = ceil_div_i(kv, 16);
+    const uint32_t stage_addr = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
 #pragma unroll
-      for (int ci = 0; ci < kMaxCombosPerWarp; ++ci) {
-        const int combo = warp + ci * (kBgmvThreads / 32);
-        if (combo < combos) {
-          const int rt = combo / NTt;
-          const int nt = combo - rt * NTt;
-          const int i = rt / tps;
-          const int r0 = (rt - i * tps) * 16;
-          const uint32_t a_addr =
-              stage_addr + (uint32_t)(i * Rpad + r0 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
-          const uint32_t x_addr = stage_addr +
-                                  (uint32_t)(L.srp + nt * 8 + (lane & 7)) * kRowStride +
-                                  ((lane >> 3) & 1) * 16;
-          for (int ks = 0; ks < nks; ++ks) {
-            uint32_t a0, a1, a2, a3, b0, b1;
-            ldsm_x4(a_addr + ks * 32, a0, a1, a2, a3);
-            ldsm_x2(x_addr + ks * 32, b0, b1);
-            if (kv - ks * 16 < 16) {  // only 8 valid input features in this step
-              a2 = 0u;
-              a3 = 0u;
-              b1 = 0u;
-            }
-            mma_bf16_16816(acc[ci], a0, a1, a2, a3, b0, b1);
+    for (int ci = 0; ci < kMaxCombosPerWarp; ++ci) {
+      const int combo = warp + ci * (kBgmvThreads / 32);
+      if (combo < combos) {
+        const int rt = combo / NTt;
+        const int nt = combo - rt * NTt;
+        const int i = rt / tps;
+        const int r0 = (rt - i * tps) * 16;
+        const uint32_t a_addr =
+            stage_addr + (uint32_t)((i * Rpad + r0 + (lane & 15)) * stride + (lane >> 4) * 16);
+        const uint32_t x_addr =
+            stage_addr + (uint32_t)((L.srp + nt * 8 + (lane & 7)) * stride + ((lane >> 3) & 1) * 16);
+        for (int ks = 0; ks < nks; ++ks) {
+          uint32_t a0, a1, a2, a3, b0, b1;
+          ldsm_x4(a_addr + ks * 32, a0, a1, a2, a3);
+          ldsm_x2(x_addr + ks * 32, b0, b1);
+          if (kv - ks * 16 < 16) {  // only 8 valid input features in this step
+            a2 = 0u;
+            a3 = 0u;
+            b1 = 0u;
           }
+          mma_bf16_16816(acc[ci], a0, a1, a2, a3, b0, b1);
         }
       }
     }
     __syncthreads();
-    if (warp == 0 && kb + kNST < nkb && *abort_flag == 0) issue(kb + kNST, st);
+    if (kb + p.nst < G.nkb) {
+      issue_rows(p, L, sm, G, w, rank, kb + p.nst, st, 0, G.nrows_a + n);
+      cp_async_commit();
+    }
   }
-  kbc += (uint32_t)nkb;
 
-  // Scatter the warp tiles into hpart.
   const int g8 = lane >> 2;
   const int c4 = lane & 3;
 #pragma unroll
@@ -182,101 +195,219 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
   }
 }
 
-// Sum the kGroup partial tiles (fixed order) into this CTA's hfull.
-LORA_DEV void cluster_reduce(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                             const float* hpart, int rank, int n) {
+// Where the h of an item comes from.
+enum HSource : int { kFromCluster = 0, kFromGlobal = 1, kFromGather = 2 };
+
+// Produce h for every (token t < kTT, slice i, column r < roundup16(rank)) of
+// the item -- the value for live tokens and r < rank, 0 elsewhere -- four
+// columns per thread.  Writes the bf16 hi/lo tiles the expand MMAs read and/or
+// the fp32 global h (tokens t % kGroup == crank).  Cluster partials are summed
+// in the fixed order 0..kGroup-1, so every CTA of the cluster holds the same h.
+template <int SRC>
+LORA_DEV void produce_h(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                        const float* hpart, int w, int rank, int n, uint32_t rowmask,
+                        bool want_tiles, bool want_global, uint32_t crank) {
   const int Rpad = round_up_i(p.R, 16);
-  const int live = p.S * rank;
-  for (int e = threadIdx.x; e < n * live; e += kBgmvThreads) {
-    const int t = e / live;
-    const int q = e - t * live;
-    const int i = q / rank;
-    const int col = i * Rpad + (q - i * rank);
-    const float* src = hpart + t * L.srp + col;
-    float s = 0.f;
+  const int q4 = ceil_div_i(rank, 16) * 4;     // groups of 4 columns per slice
+  const int per_t = p.S * q4;
+  const int total = kTT * per_t;
+  for (int e = threadIdx.x; e < total; e += kBgmvThreads) {
+    const int t = e / per_t;
+    const int q = e - t * per_t;
+    const int i = q / q4;
+    const int r0 = (q - i * q4) * 4;
+    const bool row_live = t < n && ((rowmask >> t) & 1u);
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (row_live && r0 < rank) {
+      if (SRC == kFromCluster) {
+        const float* src = hpart + t * L.srp + i * Rpad + r0;
 #pragma unroll
-    for (int c = 0; c < kGroup; ++c) s += dsmem_ld_f32(dsmem_addr(src, (uint32_t)c));
-    sm.hfull[t * L.srp + col] = s;
+        for (int c = 0; c < kGroup; ++c) {
+          const float4 f = dsmem_ld_f32x4(dsmem_addr(src, (uint32_t)c));
+          v[0] += f.x; v[1] += f.y; v[2] += f.z; v[3] += f.w;
+        }
+      } else if (SRC == kFromGlobal) {
+        const float* hg = p.h + (size_t)sm.tok[t] * p.S * p.R + i * p.R + r0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = (r0 + k < rank) ? hg[k] : 0.f;
+      } else {
+        const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(p.a) +
+                                  ((size_t)w * p.S * p.R + i * p.R + r0) * p.in + sm.ids[t];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          v[k] = (r0 + k < rank) ? __bfloat162float(ab[(size_t)k * p.in]) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (r0 + k >= rank) v[k] = 0.f;
+    }
+    if (want_tiles) {
+      uint32_t hi2[2], lo2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        const float2 hf = __bfloat1622float2(h2);
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * k] - hf.x, v[2 * k + 1] - hf.y);
+        hi2[k] = *reinterpret_cast<const uint32_t*>(&h2);
+        lo2[k] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+      const int o = (i * kTT + t) * L.hst + r0;
+      *reinterpret_cast<uint2*>(sm.hhi + o) = make_uint2(hi2[0], hi2[1]);
+      *reinterpret_cast<uint2*>(sm.hlo + o) = make_uint2(lo2[0], lo2[1]);
+    }
+    if (want_global && t < n && (t % kGroup) == (int)crank) {
+      const int tk = sm.tok[t];
+      if (tk >= 0) {
+        float* hg = p.h + (size_t)tk * p.S * p.R + i * p.R + r0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (r0 + k < rank) hg[k] = v[k];
+      }
+    }
   }
 }
 
-// Expand of one item over this CTA's share of the output columns:
-// y[row, j] = bf16(y + scal * sum_{r<rank} hfull[t, i*Rpad + r] * b[w, j, r]).
-LORA_DEV void expand_part(const BgmvParams& p, const BgmvLayout& L, const Smem& sm, int w,
-                          int rank, float scal, int n, uint32_t rowmask, uint32_t crank) {
+// Zero the four B elements k0..k0+3 (bf16 pairs lo = (k0, k0+1), hi =
+// (k0+2, k0+3)) at or past the rank.
+LORA_DEV uint2 mask_rank4(uint2 v, int k0, int rank) {
+  if (k0 + 3 < rank) return v;
+  const uint32_t m0 = (k0 < rank ? 0xffffu : 0u) | (k0 + 1 < rank ? 0xffff0000u : 0u);
+  const uint32_t m1 = (k0 + 2 < rank ? 0xffffu : 0u) | (k0 + 3 < rank ? 0xffff0000u : 0u);
+  return make_uint2(v.x & m0, v.y & m1);
+}
+
+// Expand of one item over this CTA's share of the output columns with
+// m16n8k16 MMAs: D[16 columns, 8 tokens] = B[16 columns, 16 ranks] H^T.
+// MMA row m < 8 is column 2m and row m + 8 is column 2m + 1 of the tile, and
+// MMA k (2c + e) / (2c + 8 + e) is rank 4c + e / 4c + 2 + e, so each lane
+// loads 8 contiguous bytes per operand and owns a bf16 column pair of two
+// tokens.  H = hi + lo in bf16 (two MMAs, fp32 accumulate); then
+// y = bf16_rne(y + scal * D) on the live rows.
+LORA_DEV void expand_mma(const BgmvParams& p, const BgmvLayout& L, const Smem& sm, int w,
+                         int rank, float scal, int n, uint32_t rowmask, uint32_t crank) {
+  constexpr int kMT = 3;              // 16-column tiles per warp per pass
+  constexpr int kNT = kTT / 8;        // 8-token tiles
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int g = lane >> 2;
+  const int c = lane & 3;
   const int out = p.out;
-  const int Rpad = round_up_i(p.R, 16);
-  const int ochunk = round_up_i(ceil_div_i(out, kGroup), 8);
+  const int R = p.R;
+  const int ochunk = round_up_i(ceil_div_i(out, kGroup), 16);
   const int j0 = min(out, (int)crank * ochunk);
   const int j1 = min(out, j0 + ochunk);
-  const int npairs = (j1 - j0) >> 1;
-  const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(p.b) + (size_t)w * out * p.R;
+  const int mtiles = ceil_div_i(j1 - j0, 16);
+  const int ksteps = ceil_div_i(rank, 16);
+  const int ntn = ceil_div_i(n, 8);
   uint32_t* y32 = reinterpret_cast<uint32_t*>(p.y);
-  int rowoff[kTT];
+  const uint16_t* bb = reinterpret_cast<const uint16_t*>(p.b) + (size_t)w * out * R;
+  // rows (tokens) 2c and 2c+1 of every token tile
+  size_t yoff[kNT][2];
+  bool yok[kNT][2];
 #pragma unroll
-  for (int t = 0; t < kTT; ++t) rowoff[t] = (t < n && ((rowmask >> t) & 1u)) ? sm.tok[t] : -1;
+  for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = nt * 8 + 2 * c + e;
+      yok[nt][e] = t < n && ((rowmask >> t) & 1u);
+      yoff[nt][e] = yok[nt][e] ? (size_t)sm.tok[t] * out : 0;
+    }
 
-  for (int cp = threadIdx.x; cp < npairs; cp += kBgmvThreads) {
-    const int j = j0 + 2 * cp;
-    int i = 0;
-    while (i + 1 < p.S && p.slice_off[i + 1] <= j) ++i;
-    const float* hbase = sm.hfull + i * Rpad;
-    uint32_t yv[kTT];
+  for (int base = warp; base < mtiles; base += kMT * (kBgmvThreads / 32)) {
+    uint2 bl[kMT], bh[kMT];                 // columns 2g and 2g+1, ranks 4c..4c+3 (k-step 0)
+    uint32_t yv[kMT][kNT][2];
 #pragma unroll
-    for (int t = 0; t < kTT; ++t)
-      yv[t] = rowoff[t] >= 0 ? y32[((size_t)rowoff[t] * out + j) >> 1] : 0u;
-    float acc0[kTT], acc1[kTT];
+    for (int q = 0; q < kMT; ++q) {
+      const int mt = base + q * (kBgmvThreads / 32);
+      bl[q] = bh[q] = make_uint2(0u, 0u);
+      const int j = j0 + mt * 16 + 2 * g;   // this lane's column pair
+      const bool col_ok = mt < mtiles && j < j1;
+      if (col_ok && 4 * c < R) {
+        const uint16_t* brow = bb + (size_t)j * R + 4 * c;
+        bl[q] = *reinterpret_cast<const uint2*>(brow);
+        bh[q] = *reinterpret_cast<const uint2*>(brow + R);
+      }
 #pragma unroll
-    for (int t = 0; t < kTT; ++t) { acc0[t] = 0.f; acc1[t] = 0.f; }
-    const __nv_bfloat16* b0p = bb + (size_t)j * p.R;
-    for (int rc = 0; rc < rank; rc += 8) {
-      const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(b0p + rc));
-      const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(b0p + p.R + rc));
-      float bv0[8], bv1[8];
-      bv0[0] = bf16_lo(u0.x); bv0[1] = bf16_hi(u0.x); bv0[2] = bf16_lo(u0.y); bv0[3] = bf16_hi(u0.y);
-      bv0[4] = bf16_lo(u0.z); bv0[5] = bf16_hi(u0.z); bv0[6] = bf16_lo(u0.w); bv0[7] = bf16_hi(u0.w);
-      bv1[0] = bf16_lo(u1.x); bv1[1] = bf16_hi(u1.x); bv1[2] = bf16_lo(u1.y); bv1[3] = bf16_hi(u1.y);
-      bv1[4] = bf16_lo(u1.z); bv1[5] = bf16_hi(u1.z); bv1[6] = bf16_lo(u1.w); bv1[7] = bf16_hi(u1.w);
-      const int ql = min(8, rank - rc);
+      for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-      for (int t = 0; t < kTT; ++t) {
-        if (t < n) {
-          const float* hp = hbase + t * L.srp + rc;
+        for (int e = 0; e < 2; ++e)
+          yv[q][nt][e] = (col_ok && nt < ntn && yok[nt][e]) ? y32[(yoff[nt][e] + j) >> 1] : 0u;
+    }
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (q < ql) {
-              const float hv = hp[q];
-              acc0[t] = fmaf(hv, bv0[q], acc0[t]);
-              acc1[t] = fmaf(hv, bv1[q], acc1[t]);
+    for (int q = 0; q < kMT; ++q) {
+      const int mt = base + q * (kBgmvThreads / 32);
+      if (mt >= mtiles) continue;
+      const int j = j0 + mt * 16 + 2 * g;
+      const bool col_ok = j < j1;
+      // A 16-column tile holds at most two slices (slice edges are multiples
+      // of 8): one pass per slice, each lane keeping the pass of its column.
+      const int jt = j0 + mt * 16;
+      const int jl = min(jt + 15, j1 - 1);
+      int ia = 0;
+      while (ia + 1 < p.S && p.slice_off[ia + 1] <= jt) ++ia;
+      int ib = ia;
+      while (ib + 1 < p.S && p.slice_off[ib + 1] <= jl) ++ib;
+      const int my_i = (ib != ia && j >= p.slice_off[ib]) ? ib : ia;
+      float acc[kNT][4];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[nt][k] = 0.f;
+      for (int i = ia; i <= ib; ++i) {
+        float part[kNT][4];
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) part[nt][k] = 0.f;
+        for (int ks = 0; ks < ksteps; ++ks) {
+          uint2 b0 = bl[q], b1 = bh[q];
+          const int k0 = ks * 16 + 4 * c;
+          if (ks > 0) {
+            b0 = b1 = make_uint2(0u, 0u);
+            if (col_ok && k0 < R) {
+              const uint16_t* brow = bb + (size_t)j * R + k0;
+              b0 = *reinterpret_cast<const uint2*>(brow);
+              b1 = *reinterpret_cast<const uint2*>(brow + R);
+            }
+          }
+          b0 = mask_rank4(b0, k0, rank);
+          b1 = mask_rank4(b1, k0, rank);
+          const int hrow = i * kTT;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            if (nt < ntn) {
+              const int ho = (hrow + nt * 8 + g) * L.hst + k0;
+              const uint2 hh = *reinterpret_cast<const uint2*>(sm.hhi + ho);
+              const uint2 hl = *reinterpret_cast<const uint2*>(sm.hlo + ho);
+              mma_bf16_16816(part[nt], b0.x, b1.x, b0.y, b1.y, hh.x, hh.y);
+              mma_bf16_16816(part[nt], b0.x, b1.x, b0.y, b1.y, hl.x, hl.y);
+            }
+          }
+        }
+        if (i == my_i) {
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[nt][k] = part[nt][k];
+        }
+      }
+      if (col_ok) {
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          if (nt < ntn) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              if (yok[nt][e]) {
+                const uint32_t yo = yv[q][nt][e];
+                y32[(yoff[nt][e] + j) >> 1] =
+                    pack_bf16x2(fmaf(scal, acc[nt][e], bf16_lo(yo)),
+                                fmaf(scal, acc[nt][2 + e], bf16_hi(yo)));
+              }
             }
           }
         }
       }
     }
-#pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      if (rowoff[t] >= 0) {
-        const float lo = fmaf(scal, acc0[t], bf16_lo(yv[t]));
-        const float hi = fmaf(scal, acc1[t], bf16_hi(yv[t]));
-        y32[((size_t)rowoff[t] * out + j) >> 1] = pack_bf16x2(lo, hi);
-      }
-    }
-  }
-}
-
-// Write the live columns of hfull to global h (tokens t with t % kGroup == crank).
-LORA_DEV void store_h(const BgmvParams& p, const BgmvLayout& L, const Smem& sm, int rank, int n,
-                      uint32_t rowmask_any, uint32_t crank) {
-  const int Rpad = round_up_i(p.R, 16);
-  const int live = p.S * rank;
-  const int SR = p.S * p.R;
-  for (int e = threadIdx.x; e < n * live; e += kBgmvThreads) {
-    const int t = e / live;
-    if ((t % kGroup) != (int)crank || !((rowmask_any >> t) & 1u)) continue;
-    const int q = e - t * live;
-    const int i = q / rank;
-    const int r = q - i * rank;
-    p.h[(size_t)sm.tok[t] * SR + i * p.R + r] = sm.hfull[t * L.srp + i * Rpad + r];
   }
 }
 
@@ -287,9 +418,10 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
   constexpr bool kScaled = (MODE == kModeFused || MODE == kModeExpand || MODE == kModeEmbed ||
                             MODE == kModeExpert);
+  constexpr bool kExpands = kScaled;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int npref = (MODE == kModeExpert) ? p.num_experts : p.slots;
-  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R);
+  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst);
   const Smem sm = carve(smem_raw, L);
   const int tid = threadIdx.x;
 
@@ -304,13 +436,6 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
     ngroups = gridDim.x / kGroup;
   }
 
-  if (tid == 0) {
-    for (int st = 0; st < kNST; ++st) mbar_init(&sm.bars[st], 1);
-    fence_mbar_init();
-    sm.ctrl[4] = 0;
-  }
-  __syncthreads();
-
   const bool report = (blockIdx.x == 0);
   int total;
   if (MODE == kModeExpert) {
@@ -322,19 +447,18 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
                                       report);
   }
   if (kClustered) {
-    // The trip count of every loop that contains a cluster barrier comes from
-    // rank 0, so all CTAs of a cluster take the same barriers.
+    // Trip counts of loops holding a cluster barrier come from rank 0, so every
+    // CTA of a cluster takes the same barriers.
     if (tid == 0) sm.ctrl[0] = total;
     cluster_sync();
     total = dsmem_ld_s32(dsmem_addr(&sm.ctrl[0], 0));
   }
 
-  uint32_t kbc = 0;
   int hpar = 0;
   int iter = 0;
   for (int item = (int)group; item < total; item += (int)ngroups, ++iter) {
     if (MODE != kModeExpert) {
-      // ---- linear / embedding item: (slot, tile) ----
+      // ---- linear / embedding item: (slot, tile of kTT positions) ----
       const int s = find_segment(sm.prefix, p.slots, item);
       const int j = item - sm.prefix[s];
       const int p0 = p.slot_indptr[s] + j * kTT;
@@ -342,11 +466,17 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
       const int rank = p.ranks[s];
       const float scal = kScaled ? p.scalings[s] : 0.f;
       const bool emb = (MODE == kModeEmbed || MODE == kModeGather);
+      int t = -1;
+      if (tid < n && p0 + tid >= 0 && p0 + tid < p.T) t = p.token_order[p0 + tid];
+      ShrinkGeom G = {};
+      if (kClustered) {
+        // the A rows do not depend on the tokens: start them while the reads land
+        G = shrink_geom(p, rank, crank);
+        if (G.nkb > 0) issue_rows(p, L, sm, G, s, rank, 0, 0, 0, G.nrows_a);
+      }
       if (tid < kTT) {
-        int t = -1;
         int id = -1;
         if (tid < n && p0 + tid >= 0 && p0 + tid < p.T) {
-          t = p.token_order[p0 + tid];
           if (t < 0 || t >= p.T) {
             if (crank == 0) raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
             t = -1;
@@ -361,47 +491,27 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
       }
       __syncthreads();
       uint32_t tokmask = 0, idmask = 0;
-      int nvalid = 0;
 #pragma unroll
       for (int t = 0; t < kTT; ++t) {
-        if (sm.tok[t] >= 0) { tokmask |= 1u << t; ++nvalid; }
+        if (sm.tok[t] >= 0) tokmask |= 1u << t;
         if (sm.ids[t] >= 0) idmask |= 1u << t;
       }
-      const int Rpad = round_up_i(p.R, 16);
-      if (MODE == kModeFused || MODE == kModeShrink) {
+      const uint32_t rowmask = emb ? (tokmask & idmask) : tokmask;
+      if (kClustered) {
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
-        shrink_partial(p, L, sm, kbc, s, rank, n, nvalid, crank, hp);
+        shrink_partial(p, L, sm, G, s, rank, n, hp);
         cluster_sync();
-        cluster_reduce(p, L, sm, hp, rank, n);
+        produce_h<kFromCluster>(p, L, sm, hp, s, rank, n, rowmask, kExpands,
+                                MODE == kModeShrink, crank);
         hpar ^= 1;
-        __syncthreads();
+      } else if (MODE == kModeExpand) {
+        produce_h<kFromGlobal>(p, L, sm, nullptr, s, rank, n, rowmask, true, false, crank);
       } else {
-        // gather or load h for every live column of every token of the item
-        const int live = p.S * rank;
-        for (int e = tid; e < n * live; e += kBgmvThreads) {
-          const int t = e / live;
-          const int q = e - t * live;
-          const int i = q / rank;
-          const int r = q - i * rank;
-          float v = 0.f;
-          if (MODE == kModeExpand) {
-            if ((tokmask >> t) & 1u) v = p.h[(size_t)sm.tok[t] * p.S * p.R + i * p.R + r];
-          } else {
-            if ((idmask >> t) & 1u) {
-              const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(p.a);
-              v = __bfloat162float(ab[((size_t)s * p.S * p.R + i * p.R + r) * p.in + sm.ids[t]]);
-            }
-          }
-          sm.hfull[t * L.srp + i * Rpad + r] = v;
-        }
-        __syncthreads();
+        produce_h<kFromGather>(p, L, sm, nullptr, s, rank, n, rowmask, kExpands,
+                               MODE == kModeGather, crank);
       }
-      if (MODE == kModeShrink || MODE == kModeGather) {
-        store_h(p, L, sm, rank, n, tokmask, crank);
-      } else {
-        const uint32_t rowmask = (MODE == kModeEmbed) ? (tokmask & idmask) : tokmask;
-        expand_part(p, L, sm, s, rank, scal, n, rowmask, crank);
-      }
+      __syncthreads();
+      if (kExpands) expand_mma(p, L, sm, s, rank, scal, n, rowmask, crank);
       __syncthreads();
     } else {
       // ---- MoE item: chunk of one expert's rows, split by slot ----
@@ -421,16 +531,16 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
           if (q >= m) continue;
           const int rho = start + q;
           if (rho < 0 || rho >= p.T) continue;
-          const int s = p.row_slot[rho];
-          if (s == -1) continue;
-          if (s < -1 || s >= p.slots) { bad |= LORA_FLAG_BAD_SLOT; continue; }
-          const int pi = p.pair_index[(size_t)s * E + e];
+          const int sl = p.row_slot[rho];
+          if (sl == -1) continue;
+          if (sl < -1 || sl >= p.slots) { bad |= LORA_FLAG_BAD_SLOT; continue; }
+          const int pi = p.pair_index[(size_t)sl * E + e];
           if (pi == -1) continue;
           if (pi < -1 || pi >= p.num_pairs) { bad |= LORA_FLAG_BAD_PAIR; continue; }
-          const int r = p.ranks[s];
+          const int r = p.ranks[sl];
           if (r < 0 || r > p.R) { bad |= LORA_FLAG_BAD_RANK; continue; }
-          if (r == 0 || p.scalings[s] == 0.0f) continue;
-          rs[q] = s;
+          if (r == 0 || p.scalings[sl] == 0.0f) continue;
+          rs[q] = sl;
           rp[q] = pi;
         }
         // sub-batches in ascending slot order, rows in row order
@@ -463,21 +573,23 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
       const int nsub = dsmem_ld_s32(dsmem_addr(nsub_slot, 0));
       for (int q = 0; q < nsub; ++q) {
         const bool mine = q < my_nsub;
-        const int s = mine ? sm.sub_s[q] : 0;
+        const int sl = mine ? sm.sub_s[q] : 0;
         const int w = mine ? sm.sub_p[q] : 0;
         const int n = mine ? sm.sub_cnt[q] : 0;
-        const int rank = mine ? p.ranks[s] : 0;
-        const float scal = mine ? p.scalings[s] : 0.f;
+        const int rank = mine ? p.ranks[sl] : 0;
+        const float scal = mine ? p.scalings[sl] : 0.f;
+        const ShrinkGeom G = shrink_geom(p, rank, crank);
+        if (G.nkb > 0 && rank > 0) issue_rows(p, L, sm, G, w, rank, 0, 0, 0, G.nrows_a);
         if (tid < kTT) sm.tok[tid] = (tid < n) ? sm.sub_rows[q * kTT + tid] : -1;
         __syncthreads();
         const uint32_t mask = (n >= 32) ? 0xffffffffu : ((1u << n) - 1u);
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
-        shrink_partial(p, L, sm, kbc, w, rank, n, n, crank, hp);
+        shrink_partial(p, L, sm, G, w, rank, n, hp);
         cluster_sync();
-        cluster_reduce(p, L, sm, hp, rank, n);
+        produce_h<kFromCluster>(p, L, sm, hp, w, rank, n, mask, true, false, crank);
         hpar ^= 1;
         __syncthreads();
-        expand_part(p, L, sm, w, rank, scal, n, mask, crank);
+        expand_mma(p, L, sm, w, rank, scal, n, mask, crank);
         __syncthreads();
       }
     }
@@ -502,11 +614,13 @@ LaunchCacheEntry g_cache[64];
 int g_cache_n = 0;
 
 template <int MODE>
-cudaError_t launch_mode(const BgmvParams& p, int max_items, cudaStream_t stream,
+cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stream,
                         const char** why) {
+  BgmvParams p = p_in;
+  bgmv_pick_stages(p.in, p.S, p.R, &p.kb, &p.nst);
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
   const int npref = (MODE == kModeExpert) ? p.num_experts : p.slots;
-  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R);
+  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst);
   auto kern = bgmv_kernel<MODE>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);

@@ -118,6 +118,19 @@ LORA_DEV void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------
+// 16-byte asynchronous copies global -> shared (per-thread groups)
+// ---------------------------------------------------------------------------
+
+LORA_DEV void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+LORA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+LORA_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters
 // ---------------------------------------------------------------------------
 
@@ -151,6 +164,14 @@ LORA_DEV uint32_t dsmem_addr(const void* local, uint32_t rank) {
 LORA_DEV float dsmem_ld_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+LORA_DEV float4 dsmem_ld_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
   return v;
 }
 LORA_DEV int dsmem_ld_s32(uint32_t addr) {

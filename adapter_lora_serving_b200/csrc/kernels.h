@@ -17,13 +17,12 @@ namespace lora {
 // ---------------------------------------------------------------------------
 
 constexpr int kBgmvThreads = 256;
-constexpr int kTT = 16;          // tokens (sorted rows) per work item
+constexpr int kTT = 32;          // tokens (sorted rows) per work item
 constexpr int kGroup = 8;        // CTAs per work item (cluster size)
-constexpr int kKB = 64;          // input features per pipeline stage
-constexpr int kNST = 4;          // pipeline stages
-constexpr int kRowStride = 144;  // bytes per staged row: 64 bf16 + 16 bytes of padding
-constexpr int kMaxCombosPerWarp = 4;  // (16-row tile, 8-token tile) pairs per warp
-constexpr int kMaxSRp = 256;     // num_slices * roundup(R, 16) limit of this regime
+constexpr int kMaxKB = 512;      // input features per pipeline stage (upper bound)
+constexpr int kRingBudget = 120 * 1024;  // shared-memory bytes for the staging ring
+constexpr int kMaxCombosPerWarp = 8;  // (16-row tile, 8-token tile) pairs per warp
+constexpr int kMaxSRp = 128;     // num_slices * roundup(R, 16) limit of this regime
 
 enum BgmvMode : int {
   kModeFused = 0,   // shrink + expand (apply_linear)
@@ -57,6 +56,8 @@ struct BgmvParams {
   int out;
   int num_experts;
   int num_pairs;
+  int kb;         // input features per stage (multiple of 8)
+  int nst;        // stages in the ring (1 or 2)
   int slice_off[LORA_MAX_SLICES + 1];
 };
 
@@ -65,9 +66,12 @@ struct BgmvLayout {
   int misc_off;
   int ring_off;
   int hpart_off;
-  int hfull_off;
+  int hhi_off;      // bf16 [S][kTT][hst]: h rounded to bf16
+  int hlo_off;      // bf16 [S][kTT][hst]: h - hi rounded to bf16
+  int hst;          // row stride of the bf16 h tiles (elements): roundup(R,16) + 8
   int total;
   int srp;          // S * roundup(R, 16): h row stride in shared memory (floats)
+  int row_stride;   // bytes per staged row: kb bf16 + 16 bytes of padding
   int stage_bytes;  // bytes per pipeline stage
 };
 
@@ -78,10 +82,15 @@ __host__ __device__ inline int round_up_i(int a, int b) { return ceil_div_i(a, b
 // sub_s[kTT], sub_p[kTT], sub_cnt[kTT], sub_rows[kTT*kTT].
 constexpr int kMiscInts = kTT + kTT + 8 + 8 + 3 * kTT + kTT * kTT;
 
-__host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, int R) {
+// Input features each CTA of a cluster reduces over (multiple of 8).
+__host__ __device__ inline int bgmv_kchunk(int in) { return round_up_i(ceil_div_i(in, kGroup), 8); }
+
+__host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, int R, int kb,
+                                                  int nst) {
   BgmvLayout L;
   L.srp = S * round_up_i(R, 16);
-  L.stage_bytes = (L.srp + kTT) * kRowStride;
+  L.row_stride = kb * 2 + 16;
+  L.stage_bytes = round_up_i((L.srp + kTT) * L.row_stride, 128);
   int off = 128;  // mbarriers
   L.prefix_off = off;
   off += round_up_i((npref + 1) * 4, 128);
@@ -89,13 +98,32 @@ __host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, in
   off += round_up_i(kMiscInts * 4, 128);
   L.ring_off = off;
   const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpert);
-  if (ring) off += kNST * L.stage_bytes;
+  if (ring) off += nst * L.stage_bytes;
   L.hpart_off = off;
   if (ring) off += 2 * kTT * L.srp * 4;
-  L.hfull_off = off;
-  off += kTT * L.srp * 4;
+  L.hst = round_up_i(R, 16) + 8;
+  L.hhi_off = off;
+  off += round_up_i(S * kTT * L.hst * 2, 128);
+  L.hlo_off = off;
+  off += round_up_i(S * kTT * L.hst * 2, 128);
   L.total = off;
   return L;
+}
+
+// Stage width and depth of the staging ring for these shapes (host side).
+inline void bgmv_pick_stages(int in, int S, int R, int* kb, int* nst) {
+  const int kchunk = bgmv_kchunk(in);
+  const int rows = S * round_up_i(R, 16) + kTT;
+  int k = kchunk < kMaxKB ? kchunk : kMaxKB;
+  for (;;) {
+    const int n = ceil_div_i(kchunk, k) > 1 ? 2 : 1;
+    if (k <= 64 || n * rows * (2 * k + 16) <= kRingBudget) {
+      *kb = k;
+      *nst = n;
+      return;
+    }
+    k -= 64;
+  }
 }
 
 // Launchers (bgmv.cu).  Return a cudaError_t from the launch.

@@ -526,6 +526,8 @@ def main():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-workload table")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--profile", action="store_true",
+                    help="timed steps only (no e2e, CPU baseline or table): for ncu captures")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -572,7 +574,7 @@ def main():
                 "kernel": kname or "bgmv_kernel",
                 "per_launch_us": round(kernel_s * 1e6, 3) if kernel_s else None}
 
-    e2e = time_e2e(torch, wl, args.e2e_steps) if rank == 0 else None
+    e2e = time_e2e(torch, wl, args.e2e_steps) if rank == 0 and not args.profile else None
 
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
@@ -587,12 +589,12 @@ def main():
            "roofline": roofline, "clocks": clocks,
            "gpu_launches": args.steps * wl.launches_per_step, "e2e": e2e}
 
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.profile:
         rate, sample, el = time_oracle(name, wl.host_sets[0])
         out["cpu_baseline"] = {"value": round(rate, 2), "unit": "tokens/s",
                                "cores": cpu_threads(), "kind": "oracle",
                                "sample": f"{sample} ({el:.1f} s, fp64 numpy oracle)"}
-    if rank == 0 and world == 1 and not args.no_configs:
+    if rank == 0 and world == 1 and not (args.no_configs or args.profile):
         out["configs"] = config_table(torch, L, name, wl, sec / args.steps, hbm_peak)
     if dist is not None:
         dist.barrier()

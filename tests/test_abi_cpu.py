@@ -111,8 +111,8 @@ def test_status_strings(lib):
 
 
 def test_host_queries(lib):
-    assert L.lora_plan_tile(L.LORA_OP_APPLY_LINEAR, L.LORA_REGIME_BGMV) == 16
-    assert L.lora_plan_tile(L.LORA_OP_EXPERT_APPLY, L.LORA_REGIME_AUTO) == 16
+    assert L.lora_plan_tile(L.LORA_OP_APPLY_LINEAR, L.LORA_REGIME_BGMV) == 32
+    assert L.lora_plan_tile(L.LORA_OP_EXPERT_APPLY, L.LORA_REGIME_AUTO) == 32
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
                                   L.LORA_REGIME_BGMV) == 0
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == L.LORA_REGIME_BGMV

@@ -59,6 +59,7 @@ SHAPES = [
     (50, 1032, (136,), 5, 32, 0.3),         # R=32, k split ragged across the cluster
     (33, 256, (128, 128), 2, 64, 0.0),      # R=64, two slices
     (300, 64, (8, 8, 8), 7, 8, 0.5),        # many sparse slots
+    (90, 128, (24, 40, 8), 3, 16, 0.1),     # 16-column tiles straddling slice edges
 ]
 
 
