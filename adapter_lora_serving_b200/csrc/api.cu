@@ -89,11 +89,12 @@ lora_status check_ptrs(const char* op, std::initializer_list<std::pair<const voi
 
 bool bgmv_fits(int S, int R) { return S * lora::round_up_i(R, 16) <= lora::kMaxSRp; }
 
-int resolve(int regime, int op, int T, int slots, int R, int S) {
+int resolve(int regime, int op, int T, int slots, int R, int S, int in_features = 1 << 30) {
   if (regime == LORA_REGIME_BGMV || regime == LORA_REGIME_SGMV) return regime;
-  (void)op;
+  const bool needs_shrink = (op == LORA_OP_SHRINK || op == LORA_OP_APPLY_LINEAR);
   // Many tokens per slot on average: tensor-core tiles over slot segments.
-  if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024)
+  if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024 &&
+      (!needs_shrink || in_features >= 64))
     return LORA_REGIME_SGMV;
   return LORA_REGIME_BGMV;
 }
@@ -157,7 +158,7 @@ lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* r
   if (st != LORA_OK) return st;
   if (err_flags != nullptr && !aligned4(err_flags))
     return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
-  const int reg = resolve(regime, LORA_OP_SHRINK, T, slots, R, num_slices);
+  const int reg = resolve(regime, LORA_OP_SHRINK, T, slots, R, num_slices, in_features);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
@@ -165,7 +166,7 @@ lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* r
     const char* why = nullptr;
     cudaError_t err = lora::sgmv_shrink_launch(x, a, h, ranks, token_order, slot_indptr, T,
                                                in_features, slots, R, num_slices, err_flags, s,
-                                               &why);
+                                               &why, 1, nullptr);
     if (err != cudaSuccess) return cuda_fail(err, op, why);
     return ok();
   }
@@ -206,7 +207,7 @@ lora_status lora_expand(void* y, const float* h, const void* b, const int32_t* r
     if (!lora::sgmv_supported(num_slices, R))
       return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
     const char* why = nullptr;
-    cudaError_t err = lora::sgmv_expand_launch(y, h, nullptr, nullptr, b, ranks, scalings,
+    cudaError_t err = lora::sgmv_expand_launch(y, h, 1, nullptr, nullptr, b, ranks, scalings,
                                                token_order, slot_indptr, T, 0, slots, R,
                                                num_slices, p.slice_off, out, err_flags, s, &why);
     if (err != cudaSuccess) return cuda_fail(err, op, why);
@@ -245,7 +246,7 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
   if (st != LORA_OK) return st;
   if (err_flags != nullptr && !aligned4(err_flags))
     return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
-  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, num_slices);
+  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, in_features);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
@@ -258,13 +259,14 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
       return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
     float* hws = static_cast<float*>(workspace);
     const char* why = nullptr;
+    const int ks = lora::sgmv_shrink_splits(T, slots, in_features);
     cudaError_t err = lora::sgmv_shrink_launch(x, a, hws, ranks, token_order, slot_indptr, T,
                                                in_features, slots, R, num_slices, err_flags, s,
-                                               &why);
+                                               &why, ks, scalings);
     if (err != cudaSuccess) return cuda_fail(err, op, why);
-    err = lora::sgmv_expand_launch(y, hws, nullptr, nullptr, b, ranks, scalings, token_order,
+    err = lora::sgmv_expand_launch(y, hws, ks, nullptr, nullptr, b, ranks, scalings, token_order,
                                    slot_indptr, T, 0, slots, R, num_slices, p.slice_off, out,
-                                   nullptr, s, &why);
+                                   err_flags, s, &why);
     if (err != cudaSuccess) return cuda_fail(err, op, why);
     return ok();
   }
@@ -338,9 +340,9 @@ lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, con
     if (!lora::sgmv_supported(num_slices, R))
       return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
     const char* why = nullptr;
-    cudaError_t err = lora::sgmv_expand_launch(y, nullptr, ids, a, b, ranks, scalings, token_order,
-                                               slot_indptr, T, vocab, slots, R, num_slices,
-                                               p.slice_off, out, err_flags, s, &why);
+    cudaError_t err = lora::sgmv_expand_launch(y, nullptr, 1, ids, a, b, ranks, scalings,
+                                               token_order, slot_indptr, T, vocab, slots, R,
+                                               num_slices, p.slice_off, out, err_flags, s, &why);
     if (err != cudaSuccess) return cuda_fail(err, op, why);
     return ok();
   }

@@ -10,18 +10,26 @@ namespace lora {
 
 constexpr int kSgmvTileM = 128;  // positions (tokens) per work item
 
+// Shapes the SGMV kernels take: R in {16, 32, 64}, num_slices * R <= 128.
 bool sgmv_supported(int S, int R);
+// Workspace of lora_apply_linear in this regime (partial h buffers).
 size_t sgmv_workspace_bytes(int T, int R, int S);
+// Splits of the input features the shrink uses for these shapes.
+int sgmv_shrink_splits(int T, int slots, int in);
 
-// h[t, i*R + r] = x[t] . a[slot, i*R + r] for the live columns of live tokens.
+// h[ks][t, i*R + r] = x[t, k-range ks] . a[slot, i*R + r, k-range ks] for the
+// live columns of live tokens; ksplit = min(ksplit_max, sgmv_shrink_splits()).
+// scalings == nullptr plans every slot of nonzero rank; otherwise slots of
+// scaling 0 are skipped too.
 cudaError_t sgmv_shrink_launch(const void* x, const void* a, float* h, const int* ranks,
                                const int* token_order, const int* slot_indptr, int T, int in,
                                int slots, int R, int S, uint32_t* flags, cudaStream_t stream,
-                               const char** why);
+                               const char** why, int ksplit_max, const float* scalings);
 
-// y += scal * h B^T.  h comes from `h` (fp32 [T, S*R]) or, when h is null,
-// is gathered from `a` at `ids` (embedding target, vocab columns).
-cudaError_t sgmv_expand_launch(void* y, const float* h, const int* ids, const void* a,
+// y += scal * h B^T, h = sum of `ksplit` partial buffers of `h` (fp32
+// [ksplit][T][S*R]) or, when h is null, gathered from `a` at `ids`
+// (embedding target, `vocab` columns).
+cudaError_t sgmv_expand_launch(void* y, const float* h, int ksplit, const int* ids, const void* a,
                                const void* b, const int* ranks, const float* scalings,
                                const int* token_order, const int* slot_indptr, int T, int vocab,
                                int slots, int R, int S, const int* slice_off, int out,

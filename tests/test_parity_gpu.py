@@ -13,7 +13,19 @@ from gpu_util import (LinearDev, MoEDev, assert_close, assert_rows_bit_identical
 
 pytestmark = pytest.mark.gpu
 
-REGIMES = [L.LORA_REGIME_BGMV]
+REGIMES = [pytest.param(L.LORA_REGIME_BGMV, id="bgmv"),
+           pytest.param(L.LORA_REGIME_SGMV, id="sgmv")]
+
+
+def _skip_unsupported(p, regime, shrink=True):
+    """The SGMV kernels take R in {16, 32, 64}, num_slices * R <= 128 and (for the
+    shrink) in_features >= 64; other shapes are the BGMV regime's."""
+    if regime != L.LORA_REGIME_SGMV:
+        return
+    if p.R not in (16, 32, 64) or p.num_slices * p.R > 128:
+        pytest.skip("shape outside the SGMV regime")
+    if shrink and p.n_in < 64:
+        pytest.skip("in_features < 64 is outside the SGMV shrink")
 
 
 def _f64(bits):
@@ -28,6 +40,7 @@ def _oracle_linear(p, y_bits=None, token_order=None):
 
 
 def _check_linear(p, regime, y_bits=None, what=""):
+    _skip_unsupported(p, regime)
     d = LinearDev(p, y_bits)
     d.apply_linear(regime)
     y_in = p.y if y_bits is None else y_bits
@@ -72,6 +85,24 @@ def test_random_linear(regime, shape, seed):
     _check_linear(p, regime, what=f"{shape}")
 
 
+SGMV_SHAPES = [
+    # T, in, out_slices, slots, R, ranks
+    (700, 256, (136, 64), 3, 16, [16, 8, 12]),       # 3+ tiles per slot, ragged chunks
+    (520, 192, (256,), 2, 32, [32, 20]),            # R=32 (64-byte rows)
+    (400, 128, (128, 128), 3, 64, [64, 16, 40]),    # R=64, two slices
+    (300, 64, (24, 40, 8), 2, 16, [16, 16]),        # chunks straddling slice edges
+]
+
+
+@pytest.mark.parametrize("regime", REGIMES)
+@pytest.mark.parametrize("shape", SGMV_SHAPES)
+def test_tile_shapes(regime, shape):
+    T, n_in, outs, slots, R, ranks = shape
+    p = W.random_linear(200 + T, T, n_in, outs, slots, R, ranks=ranks, dead_frac=0.05)
+    _check_linear(p, regime, what=f"{shape}")
+    _check_linear(p, regime, y_bits=np.zeros_like(p.y), what=f"{shape} y=0")
+
+
 @pytest.mark.parametrize("regime", REGIMES)
 def test_delta_visible_with_zero_y(regime):
     for p in (W.tiny_linear(1), W.random_linear(7, 80, 256, (32, 16), 4, 16, dead_frac=0.1)):
@@ -83,6 +114,7 @@ def test_delta_visible_with_zero_y(regime):
 def test_noops_bit_exact_and_poison_ignored(regime):
     p = W.random_linear(11, 90, 128, (16, 16), 5, 16, ranks=[0, 8, 16, 5, 16],
                         scalings=[1.0, 0.0, 0.5, 2.0, 1.0], dead_frac=0.2)
+    _skip_unsupported(p, regime)
     y = p.y.copy()
     y[:, 0] = 0x8000          # -0.0
     y[:, 1] = 0x7FC1          # NaN payload
@@ -105,6 +137,7 @@ def test_noops_bit_exact_and_poison_ignored(regime):
 @pytest.mark.parametrize("regime", REGIMES)
 def test_position_permutation_and_rerun_bit_exact(regime):
     p = W.random_linear(12, 120, 256, (32,), 3, 16, ranks=[16, 8, 16])
+    _skip_unsupported(p, regime)
     d = LinearDev(p)
     d.apply_linear(regime)
     first = host_bits(d.y)
@@ -125,6 +158,7 @@ def test_position_permutation_and_rerun_bit_exact(regime):
 def test_shrink_and_expand(regime):
     t = torch()
     p = W.random_linear(13, 70, 320, (24, 40), 4, 16, ranks=[16, 8, 0, 12], dead_frac=0.1)
+    _skip_unsupported(p, regime)
     d = LinearDev(p)
     SR = p.num_slices * p.R
     h = t.full((p.T, SR), float("nan"), dtype=t.float32, device="cuda")
@@ -172,6 +206,7 @@ def test_gather_shrink_exact():
 def test_apply_embedding(regime, seed):
     p = W.random_linear(15 + seed, 150, None, (64, 32), 5, 16, embedding_vocab=3000,
                         bad_id_frac=0.1, dead_frac=0.05)
+    _skip_unsupported(p, regime, shrink=False)
     d = LinearDev(p)
     d.apply_embedding(regime)
     y_ref, touched, flags = O.apply_embedding(p.ids, _f64(p.y), _f64(p.a), _f64(p.b),
@@ -244,15 +279,16 @@ def test_plan_expert_bit_exact():
 
 @pytest.mark.parametrize("regime", REGIMES)
 def test_bad_addressing_flags(regime):
-    p = W.random_linear(16, 40, 64, (16,), 4, 8, ranks=[8, 8, 8, 8])
+    p = W.random_linear(16, 40, 64, (16,), 4, 16, ranks=[16, 16, 16, 16])
     to = p.token_order.copy()
     indptr = p.slot_indptr.copy()
     ranks = p.ranks.copy()
     to[indptr[0]] = 1000                     # bad token in slot 0
-    ranks[2] = 9                             # rank > R
+    ranks[2] = 17                            # rank > R
     indptr[3] = indptr[4] + 1                # slot 3: lo > hi
     q = W.LinearProblem(**{**p.__dict__, "token_order": to, "slot_indptr": indptr,
                            "ranks": ranks})
+    _skip_unsupported(q, regime)
     d = LinearDev(q)
     d.apply_linear(regime)
     y_ref, touched, flags = O.apply_linear(_f64(q.x), _f64(q.y), _f64(q.a), _f64(q.b), to,
