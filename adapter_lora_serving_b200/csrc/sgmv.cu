@@ -30,7 +30,9 @@ namespace lora {
 
 namespace {
 
-constexpr int kSgThreads = 192;   // 6 warps
+constexpr int kSgThreads = 192;   // shrink: 6 warps
+constexpr int kExThreads = 320;   // expand: 10 warps (8 epilogue warps)
+constexpr int kNY = 3;            // y staging buffers (prefetch two units ahead)
 constexpr int kTM = kSgmvTileM;   // 128 tokens per tile (MMA M)
 constexpr int kBN = 128;          // output columns per expand unit (MMA N)
 constexpr int kNB = 4;            // B ring stages (expand)
@@ -126,7 +128,7 @@ LORA_DEV ExpandUnit expand_unit(const ExpandParams& p, const int* prefix, long l
 // Expand
 // ---------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(kSgThreads, 1)
+__global__ void __launch_bounds__(kExThreads, 1)
 sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParams p) {
   extern __shared__ uint8_t sg_smem_raw[];
   const uint32_t raw = smem_u32(sg_smem_raw);
@@ -160,9 +162,9 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 4);
+      mbar_init(&accempty[i], 8);   // one arrival per epilogue warp
     }
-    mbar_init(hready, 128);   // one arrival per epilogue thread
+    mbar_init(hready, 256);   // one arrival per epilogue thread
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmap_b);
@@ -171,7 +173,7 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     tmem_alloc(tmem_slot, 2 * kBN);
     tmem_relinquish();
   }
-  const int items = plan_linear<kSgThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
+  const int items = plan_linear<kExThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
                                             p.R, kTM, prefix, scratch, p.flags,
                                             blockIdx.x == 0);
   tc_fence_before();
@@ -242,43 +244,66 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
       __syncwarp();
     }
   } else {
-    // ---------------- epilogue: warps 2..5, one TMEM lane (token row) each ----------------
+    // ---------------- epilogue: warps 2..9 ----------------
+    // Warp w reads TMEM lanes 32*(w%4).. (one token row per thread) and owns
+    // half of the unit's 128 columns.
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int m = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    uint32_t* y32 = reinterpret_cast<uint32_t*>(p.y);
     const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(p.y);
-    int hcount = 0;
+    uint8_t* ybytes = reinterpret_cast<uint8_t*>(p.y);
     int prev_item = -1, prev_slice = -1;
-    int tok = -1;  // token of row m for the current item
 
     auto row_token = [&](const ExpandUnit& U) -> int {
       if (m >= U.n) return -1;
       const int t = p.token_order[U.p0 + m];
       return (t >= 0 && t < p.T) ? t : -1;
     };
+    // The warp's 32 rows x 64 columns of y, as 16-byte copies: lane l takes
+    // chunk l % 8 of row 4j + l / 8, so an instruction moves four full
+    // 128-byte row segments.  `t` is this lane's own row token; rows read
+    // their token from the lane that owns them.
     auto prefetch_y = [&](const ExpandUnit& U, int t, int buf) {
-      if (t >= 0) {
-        const uint32_t dst = smem_u32(ystage) + (uint32_t)(buf * kTM + m) * kYRow;
-        const __nv_bfloat16* src = yb + (size_t)t * p.out + U.col0;
-        for (int c = 0; c < (U.width >> 3); ++c) cp_async16(dst + c * 16, src + c * 8);
+      const int c = half * 8 + (lane & 7);
+      const bool cok = c < (U.width >> 3);
+      const uint32_t base_s = smem_u32(ystage) + (uint32_t)(buf * kTM + quarter * 32) * kYRow;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = 4 * j + (lane >> 3);
+        const int tr = __shfl_sync(0xffffffffu, t, r);
+        if (tr >= 0 && cok)
+          cp_async16(base_s + (uint32_t)r * kYRow + c * 16, yb + (size_t)tr * p.out + U.col0 + c * 8);
       }
       cp_async_commit();
     };
 
-    ExpandUnit U = {};
-    int tnext = -1;
-    if (nloc > 0) {
-      U = expand_unit(p, prefix, u0);
-      tnext = row_token(U);
-      prefetch_y(U, tnext, 0);
+    ExpandUnit Uq[kNY];      // units k, k+1, k+2
+    int tq[kNY];
+    for (int j = 0; j < kNY - 1; ++j) {
+      if (j < nloc) {
+        Uq[j] = expand_unit(p, prefix, u0 + j);
+        tq[j] = row_token(Uq[j]);
+        prefetch_y(Uq[j], tq[j], j);
+      } else {
+        cp_async_commit();
+      }
     }
     for (int k = 0; k < nloc; ++k) {
-      const bool new_item = U.item != prev_item;
-      if (new_item) {
-        tok = tnext;
-        if (m < U.n && tok < 0 && U.col0 == 0) raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
+      const ExpandUnit U = Uq[k % kNY];
+      const int tok = tq[k % kNY];
+      // keep two units of y in flight
+      if (k + kNY - 1 < nloc) {
+        const int j = (k + kNY - 1) % kNY;
+        Uq[j] = expand_unit(p, prefix, u0 + k + kNY - 1);
+        tq[j] = row_token(Uq[j]);
+        prefetch_y(Uq[j], tq[j], j);
+      } else {
+        cp_async_commit();
       }
+      const bool new_item = U.item != prev_item;
+      if (new_item && half == 0 && m < U.n && tok < 0 && U.col0 == 0)
+        raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
       const int rank = p.ranks[U.s];
       const float scal = p.scalings[U.s];
       bool row_ok = tok >= 0;
@@ -288,11 +313,12 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
         if (id < 0 || id >= p.vocab) row_ok = false;
       }
       if (new_item || U.slice != prev_slice) {
-        // Build H (hi and lo) for (tile, slice): MMAs of the previous unit are
-        // complete, since its epilogue waited for them.
+        // Build H (hi and lo) for (tile, slice); the MMAs of the previous unit
+        // are complete, since its epilogue waited for them.  The two warps of a
+        // row split its 16-byte chunks.
         const int Kp = ceil_div_i(rank, 16) * 16;
         const int i = U.slice;
-        for (int c8 = 0; c8 < Kp; c8 += 8) {
+        for (int c8 = half * 8; c8 < Kp; c8 += 16) {
           float v[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -324,61 +350,58 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
         }
         fence_proxy_async_smem();
         mbar_arrive(hready);
-        ++hcount;
         prev_item = U.item;
         prev_slice = U.slice;
-      }
-      // prefetch the next unit's y rows while this one computes
-      ExpandUnit Un = U;
-      if (k + 1 < nloc) {
-        Un = expand_unit(p, prefix, u0 + k + 1);
-        tnext = (Un.item == U.item) ? tok : row_token(Un);
-        prefetch_y(Un, tnext, (k + 1) & 1);
-      } else {
-        cp_async_commit();
       }
       const int as = k & 1;
       if (!warp_wait(&accfull[as], (uint32_t)((k / 2) & 1), abort_flag, p.flags)) break;
       tc_fence_after();
-      cp_async_wait<1>();
-      uint8_t* yrow = ystage + (size_t)((k & 1) * kTM + m) * kYRow;
-      const bool live = row_ok;
-      for (int cg = 0; cg < kBN / 32; ++cg) {
-        float acc[32];
-        tmem_ld_32x32(tmem_base + lane_addr + (uint32_t)(as * kBN + cg * 32), acc);
-        if (live && cg * 32 < U.width) {
+      cp_async_wait<kNY - 1>();
+      __syncwarp();   // the staged rows were copied by other lanes of this warp
+      uint8_t* ybuf = ystage + (size_t)((k % kNY) * kTM) * kYRow;
+      uint8_t* yrow = ybuf + (size_t)m * kYRow;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 yv = *reinterpret_cast<const uint4*>(yrow + cg * 64 + q * 16);
-            uint32_t w[4] = {yv.x, yv.y, yv.z, yv.w};
+      for (int cg = 0; cg < 2; ++cg) {
+        const int c0 = half * 64 + cg * 32;     // first column of this group
+        if (c0 < U.width) {                     // warp-uniform
+          float acc[32];
+          tmem_ld_32x32(tmem_base + lane_addr + (uint32_t)(as * kBN + c0), acc);
+          if (row_ok) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = q * 8 + e * 2;
-              w[e] = pack_bf16x2(fmaf(scal, acc[c], bf16_lo(w[e])),
-                                 fmaf(scal, acc[c + 1], bf16_hi(w[e])));
+            for (int q = 0; q < 4; ++q) {
+              if (c0 + q * 8 < U.width) {
+                const uint4 yv = *reinterpret_cast<const uint4*>(yrow + c0 * 2 + q * 16);
+                uint32_t w[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c = q * 8 + e * 2;
+                  w[e] = pack_bf16x2(fmaf(scal, acc[c], bf16_lo(w[e])),
+                                     fmaf(scal, acc[c + 1], bf16_hi(w[e])));
+                }
+                *reinterpret_cast<uint4*>(yrow + c0 * 2 + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
             }
-            *reinterpret_cast<uint4*>(yrow + cg * 64 + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[as]);
-      // coalesced write-back of this warp's 32 rows
-      const int wbytes = U.width * 2;
-      for (int r = 0; r < 32; ++r) {
-        const int row = quarter * 32 + r;
-        const int trow = __shfl_sync(0xffffffffu, live ? tok : -1, r);
-        if (trow < 0) continue;
-        const uint8_t* src = ystage + (size_t)((k & 1) * kTM + row) * kYRow;
-        for (int b = lane * 8; b < wbytes; b += 256) {
-          const uint2 v = *reinterpret_cast<const uint2*>(src + b);
-          *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(y32) +
-                                    ((size_t)trow * p.out + U.col0) * 2 + b) = v;
+      // coalesced write-back of the warp's 32 rows x 64 columns
+      {
+        const int c = half * 8 + (lane & 7);
+        const bool cok = c < (U.width >> 3);
+        const int tl = row_ok ? tok : -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = 4 * j + (lane >> 3);
+          const int tr = __shfl_sync(0xffffffffu, tl, r);
+          if (tr >= 0 && cok) {
+            const uint4 v = *reinterpret_cast<const uint4*>(ybuf + (size_t)(quarter * 32 + r) * kYRow + c * 16);
+            *reinterpret_cast<uint4*>(ybytes + ((size_t)tr * p.out + U.col0 + c * 8) * 2) = v;
+          }
         }
       }
-      __syncwarp();
-      U = Un;
     }
     cp_async_wait<0>();
   }
@@ -674,7 +697,7 @@ cudaError_t dev_info(DevInfo** out) {
 size_t expand_smem(int slots, int span) {
   const size_t pre = ((size_t)(slots + 1) * 4 + 1023) / 1024 * 1024;
   return 1024 + 1024 + pre + 2 * (size_t)kTM * span + (size_t)kNB * kBN * span +
-         2 * (size_t)kTM * kYRow;
+         (size_t)kNY * kTM * kYRow;
 }
 
 size_t shrink_smem(int slots) {
@@ -779,7 +802,7 @@ cudaError_t sgmv_expand_launch(void* y, const float* h, int ksplit, const int* i
   }
   const long long units = (long long)(slots + ceil_div_i(T, kTM)) * nchunk;
   const int grid = (int)max(1LL, min((long long)d->sms, units));
-  sgmv_expand_kernel<<<grid, kSgThreads, smem, stream>>>(map, p);
+  sgmv_expand_kernel<<<grid, kExThreads, smem, stream>>>(map, p);
   return cudaGetLastError();
 }
 
