@@ -100,27 +100,38 @@ LORA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag
 
 LORA_DEV uint32_t align1024(uint32_t v) { return (v + 1023u) & ~1023u; }
 
-// Work unit of the expand: tile (slot, first position, count) and column chunk.
-struct ExpandUnit {
-  int item, s, p0, n, slice, col0, width;
-};
+// Walks consecutive expand units without divisions: the item (and its slot
+// segment) is decoded only when the column chunks of an item run out.
+struct UnitCursor {
+  int item, cj, s, p0, n, slice, col0, width;
 
-LORA_DEV ExpandUnit expand_unit(const ExpandParams& p, const int* prefix, long long u) {
-  ExpandUnit U;
-  U.item = (int)(u / p.nchunk);
-  const int cj = (int)(u - (long long)U.item * p.nchunk);
-  U.s = find_segment(prefix, p.slots, U.item);
-  const int j = U.item - prefix[U.s];
-  U.p0 = p.slot_indptr[U.s] + j * kTM;
-  U.n = max(0, min(kTM, p.slot_indptr[U.s + 1] - U.p0));
-  int i = 0;
-  while (i + 1 < p.S && p.chunk_off[i + 1] <= cj) ++i;
-  U.slice = i;
-  const int c = cj - p.chunk_off[i];
-  U.col0 = p.slice_off[i] + c * kBN;
-  U.width = min(kBN, p.slice_off[i + 1] - U.col0);
-  return U;
-}
+  LORA_DEV void set_item(const ExpandParams& p, const int* prefix, int it) {
+    item = it;
+    s = find_segment(prefix, p.slots, it);
+    p0 = p.slot_indptr[s] + (it - prefix[s]) * kTM;
+    n = max(0, min(kTM, p.slot_indptr[s + 1] - p0));
+  }
+  LORA_DEV void set_chunk(const ExpandParams& p) {
+    while (slice + 1 < p.S && p.chunk_off[slice + 1] <= cj) ++slice;
+    col0 = p.slice_off[slice] + (cj - p.chunk_off[slice]) * kBN;
+    width = min(kBN, p.slice_off[slice + 1] - col0);
+  }
+  LORA_DEV void init(const ExpandParams& p, const int* prefix, long long u) {
+    const int it = (int)(u / p.nchunk);
+    cj = (int)(u - (long long)it * p.nchunk);
+    slice = 0;
+    set_item(p, prefix, it);
+    set_chunk(p);
+  }
+  LORA_DEV void advance(const ExpandParams& p, const int* prefix) {
+    if (++cj == p.nchunk) {
+      cj = 0;
+      slice = 0;
+      set_item(p, prefix, item + 1);
+    }
+    set_chunk(p);
+  }
+};
 
 }  // namespace
 
@@ -190,8 +201,9 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
   if (warp == 0) {
     // ---------------- producer: B tiles by tensor TMA ----------------
     if (lane == 0) {
-      for (int k = 0; k < nloc && !*abort_flag; ++k) {
-        const ExpandUnit U = expand_unit(p, prefix, u0 + k);
+      UnitCursor U;
+      if (nloc > 0) U.init(p, prefix, u0);
+      for (int k = 0; k < nloc && !*abort_flag; ++k, U.advance(p, prefix)) {
         const int st = k % kNB;
         if (k >= kNB &&
             !wait_or_abort(&bempty[st], (uint32_t)((k / kNB - 1) & 1), abort_flag, p.flags))
@@ -204,8 +216,9 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     // ---------------- MMA issuer ----------------
     int hcount = 0;
     int prev_item = -1, prev_slice = -1;
-    for (int k = 0; k < nloc; ++k) {
-      const ExpandUnit U = expand_unit(p, prefix, u0 + k);
+    UnitCursor U;
+    if (nloc > 0) U.init(p, prefix, u0);
+    for (int k = 0; k < nloc; ++k, U.advance(p, prefix)) {
       if (U.item != prev_item || U.slice != prev_slice) {
         if (!warp_wait(hready, (uint32_t)(hcount & 1), abort_flag, p.flags)) break;
         ++hcount;
@@ -255,49 +268,54 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     uint8_t* ybytes = reinterpret_cast<uint8_t*>(p.y);
     int prev_item = -1, prev_slice = -1;
 
-    auto row_token = [&](const ExpandUnit& U) -> int {
-      if (m >= U.n) return -1;
-      const int t = p.token_order[U.p0 + m];
+    auto row_token = [&](const UnitCursor& V) -> int {
+      if (m >= V.n) return -1;
+      const int t = p.token_order[V.p0 + m];
       return (t >= 0 && t < p.T) ? t : -1;
     };
     // The warp's 32 rows x 64 columns of y, as 16-byte copies: lane l takes
     // chunk l % 8 of row 4j + l / 8, so an instruction moves four full
     // 128-byte row segments.  `t` is this lane's own row token; rows read
     // their token from the lane that owns them.
-    auto prefetch_y = [&](const ExpandUnit& U, int t, int buf) {
+    auto prefetch_y = [&](const UnitCursor& V, int t, int buf) {
       const int c = half * 8 + (lane & 7);
-      const bool cok = c < (U.width >> 3);
+      const bool cok = c < (V.width >> 3);
       const uint32_t base_s = smem_u32(ystage) + (uint32_t)(buf * kTM + quarter * 32) * kYRow;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int r = 4 * j + (lane >> 3);
         const int tr = __shfl_sync(0xffffffffu, t, r);
         if (tr >= 0 && cok)
-          cp_async16(base_s + (uint32_t)r * kYRow + c * 16, yb + (size_t)tr * p.out + U.col0 + c * 8);
+          cp_async16(base_s + (uint32_t)r * kYRow + c * 16, yb + (size_t)tr * p.out + V.col0 + c * 8);
       }
       cp_async_commit();
     };
 
-    ExpandUnit Uq[kNY];      // units k, k+1, k+2
-    int tq[kNY];
-    for (int j = 0; j < kNY - 1; ++j) {
-      if (j < nloc) {
-        Uq[j] = expand_unit(p, prefix, u0 + j);
-        tq[j] = row_token(Uq[j]);
-        prefetch_y(Uq[j], tq[j], j);
-      } else {
-        cp_async_commit();
-      }
+    // cursors of units k, k+1, k+2 (y of the last two is in flight)
+    UnitCursor U, U1, U2;
+    int tok = -1, t1 = -1, t2 = -1;
+    if (nloc > 0) {
+      U.init(p, prefix, u0);
+      tok = row_token(U);
+      prefetch_y(U, tok, 0);
+      U1 = U;
+      U1.advance(p, prefix);
+    } else {
+      cp_async_commit();
+    }
+    if (nloc > 1) {
+      t1 = (U1.item == U.item) ? tok : row_token(U1);
+      prefetch_y(U1, t1, 1);
+      U2 = U1;
+      U2.advance(p, prefix);
+    } else {
+      cp_async_commit();
     }
     for (int k = 0; k < nloc; ++k) {
-      const ExpandUnit U = Uq[k % kNY];
-      const int tok = tq[k % kNY];
       // keep two units of y in flight
-      if (k + kNY - 1 < nloc) {
-        const int j = (k + kNY - 1) % kNY;
-        Uq[j] = expand_unit(p, prefix, u0 + k + kNY - 1);
-        tq[j] = row_token(Uq[j]);
-        prefetch_y(Uq[j], tq[j], j);
+      if (k + 2 < nloc) {
+        t2 = (U2.item == U1.item) ? t1 : row_token(U2);
+        prefetch_y(U2, t2, (k + 2) % kNY);
       } else {
         cp_async_commit();
       }
@@ -402,6 +420,11 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
           }
         }
       }
+      U = U1;
+      tok = t1;
+      U1 = U2;
+      t1 = t2;
+      if (k + 3 < nloc) U2.advance(p, prefix);
     }
     cp_async_wait<0>();
   }
