@@ -106,6 +106,11 @@ int linear_items_bound(int T, int slots, int tile) {
 
 }  // namespace
 
+namespace lora {
+// Lets other entry points of the library report through lora_last_error().
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+}  // namespace lora
+
 extern "C" {
 
 const char* lora_status_string(lora_status status) {

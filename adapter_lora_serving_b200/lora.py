@@ -39,6 +39,8 @@ LORA_OP_GATHER_SHRINK = 3
 LORA_OP_APPLY_EMBEDDING = 4
 LORA_OP_EXPERT_APPLY = 5
 
+LORA_STATIC_SCRATCH_BYTES = 16 << 20
+
 # (name, restype, argtypes) of every exported symbol.
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -48,6 +50,8 @@ _SIGS = [
     ("lora_expand", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _P, _P]),
     ("lora_apply_linear", _I,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _Z, _P, _P]),
+    ("lora_apply_linear_noalloc", _I,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _P]),
     ("lora_gather_shrink", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     ("lora_apply_embedding", _I,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _P]),
@@ -143,6 +147,18 @@ def lora_apply_linear(x, y, a, b, ranks, scalings, token_order, slot_indptr, T, 
                                     in_features, slots, R, _slices(out_slices), len(out_slices),
                                     regime, _ptr(workspace), workspace_bytes, _ptr(err_flags),
                                     _stream(stream)))
+
+
+def lora_apply_linear_noalloc(x, y, a, b, ranks, scalings, token_order, slot_indptr, T,
+                              in_features, slots, R, out_slices, regime=LORA_REGIME_AUTO,
+                              err_flags=None, stream=None):
+    """lora_apply_linear without a workspace, for callers that cannot allocate
+    device memory: the library's fixed scratch array is used instead."""
+    _check(load().lora_apply_linear_noalloc(_ptr(x), _ptr(y), _ptr(a), _ptr(b), _ptr(ranks),
+                                            _ptr(scalings), _ptr(token_order),
+                                            _ptr(slot_indptr), T, in_features, slots, R,
+                                            _slices(out_slices), len(out_slices), regime,
+                                            _ptr(err_flags), _stream(stream)))
 
 
 def lora_gather_shrink(ids, h, a, ranks, token_order, slot_indptr, T, vocab, slots, R,

@@ -192,6 +192,31 @@ LORA_API lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, con
                               uint32_t* err_flags, void* stream);
 
 /*
+ * lora_apply_linear_noalloc -- lora_apply_linear for callers that cannot give
+ * the library any device memory.  The pages have no counterpart: it exists for
+ * this library's users.  Some callers cannot allocate where they apply the
+ * delta (a plugin inside a runtime that owns all device memory and offers no
+ * allocator, code running where cudaMalloc must not be called); this entry
+ * point takes the lora_apply_linear arguments without the workspace and uses
+ * a scratch array of LORA_STATIC_SCRATCH_BYTES compiled into the library
+ * (every GPU that loads the library holds it until the process exits).
+ * Shapes whose workspace (lora_workspace_bytes) exceeds that size return
+ * LORA_ERR_UNSUPPORTED.  The first call on each device looks up the array's
+ * device address with cudaGetSymbolAddress, so make that first call outside
+ * stream capture.  It never allocates.  All calls share the array and it keeps
+ * the last call's contents (nothing needs clearing); calls that can overlap on
+ * the GPU race on it.
+ */
+#define LORA_STATIC_SCRATCH_BYTES (16u << 20)
+LORA_API lora_status lora_apply_linear_noalloc(const void* x, void* y, const void* a, const void* b,
+                                               const int32_t* ranks, const float* scalings,
+                                               const int32_t* token_order,
+                                               const int32_t* slot_indptr, int32_t T,
+                                               int32_t in_features, int32_t slots, int32_t R,
+                                               const int32_t* out_slices, int32_t num_slices,
+                                               int32_t regime, uint32_t* err_flags, void* stream);
+
+/*
  * Workspace bytes an operation needs for these shapes and regime (0 if none).
  * For LORA_OP_EXPERT_APPLY pass rows_cap as T and num_experts as slots.
  */
