@@ -141,11 +141,10 @@ int32_t lora_plan_tile(int32_t op, int32_t regime) {
 
 size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R, int32_t num_slices,
                             int32_t regime) {
-  if (op != LORA_OP_APPLY_LINEAR || T <= 0 || R <= 0 || num_slices <= 0 || slots <= 0) return 0;
+  if (op != LORA_OP_APPLY_LINEAR || T <= 0 || R <= 0 || num_slices <= 0) return 0;
   const int reg = resolve(regime, op, T, slots, R, num_slices);
-  if (reg == LORA_REGIME_SGMV)
-    return lora::kCounterReserve + lora::sgmv_workspace_bytes(T, R, num_slices);
-  return lora::bgmv_coop_workspace_bytes(T, slots, R, num_slices);
+  if (reg != LORA_REGIME_SGMV) return 0;
+  return lora::sgmv_workspace_bytes(T, R, num_slices);
 }
 
 lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* ranks,
@@ -263,7 +262,7 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
                   workspace == nullptr ? (size_t)0 : workspace_bytes);
     if (!aligned16(workspace))
       return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
-    float* hws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + lora::kCounterReserve);
+    float* hws = static_cast<float*>(workspace);
     const char* why = nullptr;
     const int ks = lora::sgmv_shrink_splits(T, slots, in_features);
     cudaError_t err = lora::sgmv_shrink_launch(x, a, hws, ranks, token_order, slot_indptr, T,
@@ -279,17 +278,12 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
   if (!bgmv_fits(num_slices, R))
     return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
                 num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
-  const size_t need = lora::bgmv_coop_workspace_bytes(T, slots, R, num_slices);
-  if (workspace == nullptr || workspace_bytes < need)
-    return fail(LORA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", op, need,
-                workspace == nullptr ? (size_t)0 : workspace_bytes);
-  if (!aligned16(workspace))
-    return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
   p.x = x; p.y = y; p.a = a; p.b = b; p.ranks = ranks; p.scalings = scalings;
   p.token_order = token_order; p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T;
   p.in = in_features; p.slots = slots; p.R = R; p.S = num_slices; p.out = out;
   const char* why = nullptr;
-  cudaError_t err = lora::bgmv_coop_launch(p, workspace, s, &why);
+  cudaError_t err = lora::bgmv_launch(lora::kModeFused, p, linear_items_bound(T, slots, lora::kTT),
+                                      s, &why);
   if (err != cudaSuccess) return cuda_fail(err, op, why);
   return ok();
 }

@@ -598,470 +598,6 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
 }
 
 // ---------------------------------------------------------------------------
-// Cooperative fused kernel (apply_linear in the BGMV regime)
-//
-// Work item = up to kTT positions of one slot.  Each item has kGroup
-// "A-units" (the shrink over one eighth of the input features; its partial h
-// goes to the workspace) and kGroup "B-units" (the expand of one eighth of the
-// output columns).  Every CTA runs its A-units first, then its B-units.  A
-// B-unit first starts the copies of its B columns and y rows into shared
-// memory, then waits (bounded) until the item's kGroup partials are in, sums
-// them in a fixed order (so results do not depend on timing) and expands.
-// The launch is cooperative: all CTAs are resident, so every A-unit runs and
-// every wait ends.  The item counters live in the workspace, start at zero and
-// are returned to zero by the last B-unit of each item.  Loops are kept rolled
-// so the kernel's code stays small enough for the instruction cache.
-// ---------------------------------------------------------------------------
-
-constexpr int kTokCache = 2048;    // token_order cached in shared memory up to this T
-
-struct CoopLayout {
-  int prefix_off, misc_off, tokc_off, soff_off, stage_off, hpart_off, hhi_off, hlo_off, total;
-  int srp, hst, arow, brow, yrow, ochunk;
-};
-
-__host__ __device__ inline CoopLayout coop_layout(int slots, int T, int S, int R, int kb,
-                                                 int out) {
-  CoopLayout L;
-  L.srp = S * round_up_i(R, 16);
-  L.hst = round_up_i(R, 16) + 8;
-  L.arow = kb * 2 + 16;                          // staged A / x row pitch
-  L.ochunk = round_up_i(ceil_div_i(out, kGroup), 16);
-  L.brow = R * 2 + 16;                           // staged B row pitch
-  L.yrow = L.ochunk * 2 + 16;                    // staged y row pitch
-  int off = 0;
-  L.prefix_off = off;
-  off += round_up_i((slots + 1) * 4, 128);
-  L.misc_off = off;
-  off += round_up_i(kMiscInts * 4, 128);
-  L.tokc_off = off;
-  off += round_up_i((T < kTokCache ? T : kTokCache) * 4, 128);
-  L.soff_off = off;
-  off += 128;
-  L.stage_off = off;
-  const int a_bytes = (L.srp + kTT) * L.arow;
-  const int b_bytes = L.ochunk * L.brow + kTT * L.yrow;
-  off += round_up_i(a_bytes > b_bytes ? a_bytes : b_bytes, 128);
-  L.hpart_off = off;
-  off += kTT * L.srp * 4;
-  L.hhi_off = off;
-  off += round_up_i(S * kTT * L.hst * 2, 128);
-  L.hlo_off = off;
-  off += round_up_i(S * kTT * L.hst * 2, 128);
-  L.total = off;
-  return L;
-}
-
-LORA_DEV int ld_acquire_gpu(const int* ptr) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
-}
-
-__global__ void __launch_bounds__(kBgmvThreads)
-bgmv_coop_kernel(const BgmvParams p, int* cnt, int* done, float* part) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  const CoopLayout L = coop_layout(p.slots, p.T, p.S, p.R, p.kb, p.out);
-  int* prefix = reinterpret_cast<int*>(smem_raw + L.prefix_off);
-  int* misc = reinterpret_cast<int*>(smem_raw + L.misc_off);
-  int* tok = misc;                      // [kTT]
-  int* ctrl = misc + 2 * kTT;
-  int* scratch = misc + 2 * kTT + 8;
-  int* tokc = reinterpret_cast<int*>(smem_raw + L.tokc_off);
-  int* soff = reinterpret_cast<int*>(smem_raw + L.soff_off);
-  uint8_t* stage = smem_raw + L.stage_off;
-  float* hpart = reinterpret_cast<float*>(smem_raw + L.hpart_off);
-  uint16_t* hhi = reinterpret_cast<uint16_t*>(smem_raw + L.hhi_off);
-  uint16_t* hlo = reinterpret_cast<uint16_t*>(smem_raw + L.hlo_off);
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int g = lane >> 2;
-  const int c = lane & 3;
-  const bool cache_tokens = p.T <= kTokCache;
-  const int Rpad = round_up_i(p.R, 16);
-
-  // Addressing: the token list travels in the same round trip as the segments.
-  if (cache_tokens)
-    for (int i = tid; i < p.T; i += kBgmvThreads) tokc[i] = p.token_order[i];
-  if (tid <= LORA_MAX_SLICES) soff[tid] = p.slice_off[tid];
-  const int items = plan_linear<kBgmvThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
-                                              p.R, kTT, prefix, scratch, p.flags,
-                                              blockIdx.x == 0);
-  const int nunits = items * kGroup;
-  const size_t tile = (size_t)kTT * L.srp;  // floats per partial tile
-
-  // Slot, first position and count of an item; its tokens go to tok[] (the
-  // caller synchronises before reading them).
-  auto load_item = [&](int item, int& s, int& n, bool report) {
-    s = find_segment(prefix, p.slots, item);
-    const int p0 = p.slot_indptr[s] + (item - prefix[s]) * kTT;
-    n = max(0, min(kTT, p.slot_indptr[s + 1] - p0));
-    if (tid < kTT) {
-      int t = -1;
-      if (tid < n && p0 + tid >= 0 && p0 + tid < p.T) {
-        t = cache_tokens ? tokc[p0 + tid] : p.token_order[p0 + tid];
-        if (t < 0 || t >= p.T) {
-          if (report) raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
-          t = -1;
-        }
-      }
-      tok[tid] = t;
-    }
-  };
-
-  // ---------------- A-units: shrink partials ----------------
-#pragma unroll 1
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-    const int item = u / kGroup;
-    const int q = u - item * kGroup;
-    int s, n;
-    load_item(item, s, n, q == 0);
-    const int rank = p.ranks[s];
-    const int kchunk = bgmv_kchunk(p.in);
-    const int k0 = min(p.in, q * kchunk);
-    const int k1 = min(p.in, k0 + kchunk);
-    const int tps = ceil_div_i(rank, 16);
-    const int NTt = ceil_div_i(n, 8);
-    const int combos = p.S * tps * NTt;
-    const __nv_bfloat16* abase =
-        reinterpret_cast<const __nv_bfloat16*>(p.a) + (size_t)s * p.S * p.R * p.in;
-    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(p.x);
-    __syncthreads();   // tok[] ready; the stage is free
-#pragma unroll 1
-    for (int kb0 = k0; kb0 < k1; kb0 += p.kb) {
-      const int kv = min(p.kb, k1 - kb0);
-      const int cpr = kv >> 3;
-      // stage the live A rows and the item's x rows (a warp per row)
-#pragma unroll 1
-      for (int i = 0; i < p.S; ++i) {
-#pragma unroll 1
-        for (int r = warp; r < rank; r += kBgmvThreads / 32) {
-          const __nv_bfloat16* src = abase + (size_t)(i * p.R + r) * p.in + kb0;
-          const uint32_t dst = smem_u32(stage) + (uint32_t)((i * Rpad + r) * L.arow);
-#pragma unroll 1
-          for (int cc = lane; cc < cpr; cc += 32) cp_async16(dst + cc * 16, src + cc * 8);
-        }
-      }
-#pragma unroll 1
-      for (int t = warp; t < n; t += kBgmvThreads / 32) {
-        const int tk = tok[t];
-        if (tk < 0) continue;
-        const __nv_bfloat16* src = xb + (size_t)tk * p.in + kb0;
-        const uint32_t dst = smem_u32(stage) + (uint32_t)((L.srp + t) * L.arow);
-#pragma unroll 1
-        for (int cc = lane; cc < cpr; cc += 32) cp_async16(dst + cc * 16, src + cc * 8);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncthreads();
-      const int nks = ceil_div_i(kv, 16);
-#pragma unroll 1
-      for (int combo = warp; combo < combos; combo += kBgmvThreads / 32) {
-        const int rt = combo / NTt;
-        const int nt = combo - rt * NTt;
-        const int i = rt / tps;
-        const int r0 = (rt - i * tps) * 16;
-        const uint32_t a_addr = smem_u32(stage) +
-            (uint32_t)((i * Rpad + r0 + (lane & 15)) * L.arow + (lane >> 4) * 16);
-        const uint32_t x_addr = smem_u32(stage) +
-            (uint32_t)((L.srp + nt * 8 + (lane & 7)) * L.arow + ((lane >> 3) & 1) * 16);
-        // two independent accumulators (even / odd k-steps) halve the MMA chain
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        float acc2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-        for (int ks = 0; ks < nks; ks += 2) {
-          uint32_t a0, a1, a2, a3, b0, b1;
-          ldsm_x4(a_addr + ks * 32, a0, a1, a2, a3);
-          ldsm_x2(x_addr + ks * 32, b0, b1);
-          if (kv - ks * 16 < 16) {
-            a2 = 0u;
-            a3 = 0u;
-            b1 = 0u;
-          }
-          mma_bf16_16816(acc, a0, a1, a2, a3, b0, b1);
-          if (ks + 1 < nks) {
-            ldsm_x4(a_addr + (ks + 1) * 32, a0, a1, a2, a3);
-            ldsm_x2(x_addr + (ks + 1) * 32, b0, b1);
-            if (kv - (ks + 1) * 16 < 16) {
-              a2 = 0u;
-              a3 = 0u;
-              b1 = 0u;
-            }
-            mma_bf16_16816(acc2, a0, a1, a2, a3, b0, b1);
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] += acc2[k];
-        const int row = i * Rpad + r0 + g;
-        const int t0 = nt * 8 + 2 * c;
-        float* h0 = hpart + t0 * L.srp + row;
-        if (kb0 == k0) {
-          h0[0] = acc[0]; h0[L.srp] = acc[1]; h0[8] = acc[2]; h0[L.srp + 8] = acc[3];
-        } else {
-          h0[0] += acc[0]; h0[L.srp] += acc[1]; h0[8] += acc[2]; h0[L.srp + 8] += acc[3];
-        }
-      }
-      __syncthreads();
-    }
-    if (k1 <= k0) {  // no input features on this split: the partial is zero
-      for (int e = tid; e < n * L.srp; e += kBgmvThreads) hpart[e] = 0.f;
-      __syncthreads();
-    }
-    float4* dst = reinterpret_cast<float4*>(part + (size_t)u * tile);
-    const float4* src = reinterpret_cast<const float4*>(hpart);
-    for (int e = tid; e < n * L.srp / 4; e += kBgmvThreads) dst[e] = src[e];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) atomicAdd(&cnt[item], 1);
-  }
-
-  // ---------------- B-units: wait for the partials, sum, expand ----------------
-  const uint16_t* bsm = reinterpret_cast<const uint16_t*>(stage);
-#pragma unroll 1
-  for (int v = blockIdx.x; v < nunits; v += gridDim.x) {
-    const int item = v / kGroup;
-    const int jc = v - item * kGroup;
-    int s, n;
-    load_item(item, s, n, false);
-    const int rank = p.ranks[s];
-    const float scal = p.scalings[s];
-    const int j0 = min(p.out, jc * L.ochunk);
-    const int j1 = min(p.out, j0 + L.ochunk);
-    const int ncol = j1 - j0;
-    __syncthreads();   // tok[] ready; the stage is free
-    // start the copies of B columns [j0, j1) and the item's y rows
-    {
-      const uint16_t* bsrc = reinterpret_cast<const uint16_t*>(p.b) +
-                             ((size_t)s * p.out + j0) * p.R;
-      const int bchunks = ncol * (p.R >> 3);
-#pragma unroll 1
-      for (int e = tid; e < bchunks; e += kBgmvThreads) {
-        const int row = e / (p.R >> 3);
-        const int cc = e - row * (p.R >> 3);
-        cp_async16(smem_u32(stage) + (uint32_t)(row * L.brow + cc * 16), bsrc + (size_t)e * 8);
-      }
-      const uint32_t ybase = smem_u32(stage) + (uint32_t)(L.ochunk * L.brow);
-      const int ychunks = ncol >> 3;
-#pragma unroll 1
-      for (int e = tid; e < n * ychunks; e += kBgmvThreads) {
-        const int t = e / ychunks;
-        const int cc = e - t * ychunks;
-        const int tk = tok[t];
-        if (tk >= 0)
-          cp_async16(ybase + (uint32_t)(t * L.yrow + cc * 16),
-                     reinterpret_cast<const uint16_t*>(p.y) + (size_t)tk * p.out + j0 + cc * 8);
-      }
-      cp_async_commit();
-    }
-    if (tid == 0) {
-      bool ok = ld_acquire_gpu(&cnt[item]) >= kGroup;
-      if (!ok) {
-        const uint64_t t0 = global_timer_ns();
-        while (!(ok = ld_acquire_gpu(&cnt[item]) >= kGroup)) {
-          if (global_timer_ns() - t0 > kWaitLimitNs) break;
-        }
-      }
-      ctrl[4] = ok ? 0 : 1;
-      if (!ok) raise_flag(p.flags, LORA_FLAG_TIMEOUT);
-    }
-    __syncthreads();
-    const bool timed_out = ctrl[4] != 0;
-    uint32_t rowmask = 0;
-#pragma unroll 1
-    for (int t = 0; t < kTT; ++t)
-      if (tok[t] >= 0) rowmask |= 1u << t;
-    // h = sum of the kGroup partials in a fixed order: fp32 in hpart for the
-    // items of at most 8 tokens (CUDA-core expand), bf16 hi + lo tiles for the
-    // larger ones (MMA expand)
-    const bool small = n <= 8;
-    const int q4 = ceil_div_i(rank, 16) * 4;
-    const int per_t = p.S * q4;
-    const float* pbase = part + (size_t)item * kGroup * tile;
-#pragma unroll 1
-    for (int e = tid; e < kTT * per_t; e += kBgmvThreads) {
-      const int t = e / per_t;
-      if (small && t >= n) break;
-      const int qq = e - t * per_t;
-      const int i = qq / q4;
-      const int r0 = (qq - i * q4) * 4;
-      float vv[4] = {0.f, 0.f, 0.f, 0.f};
-      if (!timed_out && t < n && ((rowmask >> t) & 1u) && r0 < rank) {
-        const float* src = pbase + (size_t)t * L.srp + i * Rpad + r0;
-        float4 f[kGroup];
-#pragma unroll
-        for (int qk = 0; qk < kGroup; ++qk)
-          f[qk] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)qk * tile));
-#pragma unroll
-        for (int qk = 0; qk < kGroup; ++qk) {
-          vv[0] += f[qk].x; vv[1] += f[qk].y; vv[2] += f[qk].z; vv[3] += f[qk].w;
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (r0 + k >= rank) vv[k] = 0.f;
-      }
-      if (small) {
-        *reinterpret_cast<float4*>(hpart + t * L.srp + i * Rpad + r0) =
-            make_float4(vv[0], vv[1], vv[2], vv[3]);
-        continue;
-      }
-      uint32_t hi2[2], lo2[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(vv[2 * k], vv[2 * k + 1]);
-        const float2 hf = __bfloat1622float2(h2);
-        const __nv_bfloat162 l2 = __floats2bfloat162_rn(vv[2 * k] - hf.x, vv[2 * k + 1] - hf.y);
-        hi2[k] = *reinterpret_cast<const uint32_t*>(&h2);
-        lo2[k] = *reinterpret_cast<const uint32_t*>(&l2);
-      }
-      const int o = (i * kTT + t) * L.hst + r0;
-      *reinterpret_cast<uint2*>(hhi + o) = make_uint2(hi2[0], hi2[1]);
-      *reinterpret_cast<uint2*>(hlo + o) = make_uint2(lo2[0], lo2[1]);
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    if (tid == 0 && !timed_out) {
-      // the last reader of this item's partials returns its counters to zero
-      if (atomicAdd(&done[item], 1) == kGroup - 1) {
-        cnt[item] = 0;
-        done[item] = 0;
-      }
-    }
-    if (!timed_out && small) {
-      // Expand on CUDA cores: a thread owns a column pair and loops over the
-      // item's tokens; y = bf16_rne(y + scal * sum_r h[t, r] * b[j, r]).
-      const uint8_t* ysm = stage + L.ochunk * L.brow;
-      uint32_t* y32 = reinterpret_cast<uint32_t*>(p.y);
-#pragma unroll 1
-      for (int cp = tid; cp < (ncol >> 1); cp += kBgmvThreads) {
-        const int jl = 2 * cp;
-        int i = 0;
-        while (i + 1 < p.S && soff[i + 1] <= j0 + jl) ++i;
-        const float* hcol = hpart + i * Rpad;
-        const uint8_t* b0row = stage + jl * L.brow;
-        float a0[kTT / 2], a1[kTT / 2];   // up to 8 tokens (kTT / 2 >= 8)
-#pragma unroll
-        for (int t = 0; t < 8; ++t) { a0[t] = 0.f; a1[t] = 0.f; }
-#pragma unroll 1
-        for (int r0 = 0; r0 < rank; r0 += 8) {
-          const uint4 u0 = *reinterpret_cast<const uint4*>(b0row + r0 * 2);
-          const uint4 u1 = *reinterpret_cast<const uint4*>(b0row + L.brow + r0 * 2);
-          float w0[8], w1[8];
-          w0[0] = bf16_lo(u0.x); w0[1] = bf16_hi(u0.x); w0[2] = bf16_lo(u0.y); w0[3] = bf16_hi(u0.y);
-          w0[4] = bf16_lo(u0.z); w0[5] = bf16_hi(u0.z); w0[6] = bf16_lo(u0.w); w0[7] = bf16_hi(u0.w);
-          w1[0] = bf16_lo(u1.x); w1[1] = bf16_hi(u1.x); w1[2] = bf16_lo(u1.y); w1[3] = bf16_hi(u1.y);
-          w1[4] = bf16_lo(u1.z); w1[5] = bf16_hi(u1.z); w1[6] = bf16_lo(u1.w); w1[7] = bf16_hi(u1.w);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (r0 + q >= rank) { w0[q] = 0.f; w1[q] = 0.f; }
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            if (t < n) {
-              const float4 h0 = *reinterpret_cast<const float4*>(hcol + t * L.srp + r0);
-              const float4 h1 = *reinterpret_cast<const float4*>(hcol + t * L.srp + r0 + 4);
-              const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                a0[t] = fmaf(hv[q], w0[q], a0[t]);
-                a1[t] = fmaf(hv[q], w1[q], a1[t]);
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (t < n && ((rowmask >> t) & 1u)) {
-            const uint32_t yo = *reinterpret_cast<const uint32_t*>(ysm + t * L.yrow + jl * 2);
-            y32[((size_t)tok[t] * p.out + j0 + jl) >> 1] =
-                pack_bf16x2(fmaf(scal, a0[t], bf16_lo(yo)), fmaf(scal, a1[t], bf16_hi(yo)));
-          }
-        }
-      }
-    } else if (!timed_out) {
-      // Expand: D[16 columns, 8 tokens] = B[16, rank] H^T per m16n8k16 MMA, with
-      // MMA row m < 8 = column 2m and row m + 8 = column 2m + 1 of the tile and
-      // MMA k (2c + e) / (2c + 8 + e) = rank 4c + e / 4c + 2 + e, so each lane
-      // reads 8 contiguous bytes per operand and owns a column pair of 2 tokens.
-      const int ksteps = ceil_div_i(rank, 16);
-      const int ntn = ceil_div_i(n, 8);
-      const int mtiles = ceil_div_i(ncol, 16);
-      const uint8_t* ysm = stage + L.ochunk * L.brow;
-      uint32_t* y32 = reinterpret_cast<uint32_t*>(p.y);
-#pragma unroll 1
-      for (int mt = warp; mt < mtiles; mt += kBgmvThreads / 32) {
-        const int jl = mt * 16 + 2 * g;          // column pair within the chunk
-        const bool col_ok = jl < ncol;
-        const int jt = j0 + mt * 16;
-        const int jlast = min(jt + 15, j1 - 1);
-        int ia = 0;
-        while (ia + 1 < p.S && soff[ia + 1] <= jt) ++ia;
-        int ib = ia;
-        while (ib + 1 < p.S && soff[ib + 1] <= jlast) ++ib;
-        const int my_i = (ib != ia && j0 + jl >= soff[ib]) ? ib : ia;
-        float acc[kTT / 8][4];
-#pragma unroll
-        for (int nt = 0; nt < kTT / 8; ++nt)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[nt][k] = 0.f;
-#pragma unroll 1
-        for (int i = ia; i <= ib; ++i) {
-          float part_acc[kTT / 8][4];
-#pragma unroll
-          for (int nt = 0; nt < kTT / 8; ++nt)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) part_acc[nt][k] = 0.f;
-#pragma unroll 1
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const int k0 = ks * 16 + 4 * c;
-            uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
-            if (col_ok && k0 < p.R) {
-              b0 = *reinterpret_cast<const uint2*>(bsm + ((jl * L.brow) >> 1) + k0);
-              b1 = *reinterpret_cast<const uint2*>(bsm + (((jl + 1) * L.brow) >> 1) + k0);
-            }
-            b0 = mask_rank4(b0, k0, rank);
-            b1 = mask_rank4(b1, k0, rank);
-#pragma unroll
-            for (int nt = 0; nt < kTT / 8; ++nt) {
-              if (nt < ntn) {
-                const int ho = (i * kTT + nt * 8 + g) * L.hst + k0;
-                const uint2 hh = *reinterpret_cast<const uint2*>(hhi + ho);
-                const uint2 hl = *reinterpret_cast<const uint2*>(hlo + ho);
-                mma_bf16_16816(part_acc[nt], b0.x, b1.x, b0.y, b1.y, hh.x, hh.y);
-                mma_bf16_16816(part_acc[nt], b0.x, b1.x, b0.y, b1.y, hl.x, hl.y);
-              }
-            }
-          }
-          if (i == my_i) {
-#pragma unroll
-            for (int nt = 0; nt < kTT / 8; ++nt)
-#pragma unroll
-              for (int k = 0; k < 4; ++k) acc[nt][k] = part_acc[nt][k];
-          }
-        }
-        if (col_ok) {
-#pragma unroll
-          for (int nt = 0; nt < kTT / 8; ++nt) {
-            if (nt < ntn) {
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int t = nt * 8 + 2 * c + e;
-                if (t < n && ((rowmask >> t) & 1u)) {
-                  const uint32_t yo = *reinterpret_cast<const uint32_t*>(ysm + t * L.yrow + jl * 2);
-                  y32[((size_t)tok[t] * p.out + j0 + jl) >> 1] =
-                      pack_bf16x2(fmaf(scal, acc[nt][e], bf16_lo(yo)),
-                                  fmaf(scal, acc[nt][2 + e], bf16_hi(yo)));
-                }
-              }
-            }
-          }
-        }
-      }
-    }
-    __syncthreads();
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
 
@@ -1155,81 +691,6 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
 }
 
 }  // namespace
-
-size_t bgmv_coop_workspace_bytes(int T, int slots, int R, int S) {
-  const long long items = (long long)slots + ceil_div_i(T, kTT);
-  const long long srp = (long long)S * round_up_i(R, 16);
-  return kCounterReserve + (size_t)(items * kGroup * kTT * srp * 4);
-}
-
-cudaError_t bgmv_coop_launch(const BgmvParams& p_in, void* workspace, cudaStream_t stream,
-                             const char** why) {
-  BgmvParams p = p_in;
-  // one stage of up to kMaxKB input features, as large as the shared memory allows
-  p.nst = 1;
-  p.kb = min(kMaxKB, bgmv_kchunk(p.in));
-  while (p.kb > 64 && coop_layout(p.slots, p.T, p.S, p.R, p.kb, p.out).total > 110 * 1024) p.kb -= 64;
-  const CoopLayout L = coop_layout(p.slots, p.T, p.S, p.R, p.kb, p.out);
-  const int items_max = p.slots + ceil_div_i(p.T, kTT);
-  if (2LL * items_max * 4 > kCounterReserve) {
-    *why = "too many work items for the workspace counter region";
-    return cudaErrorInvalidValue;
-  }
-  const size_t smem = (size_t)L.total;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  static std::mutex mu;
-  static int sms_cache[64] = {};
-  static bool attr_set[64] = {};
-  int sms = 0, max_optin = 0;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (sms_cache[dev] == 0) {
-      err = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
-      if (err != cudaSuccess) return err;
-    }
-    sms = sms_cache[dev];
-    err = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (err != cudaSuccess) return err;
-    if ((int)smem > max_optin) {
-      *why = "shared memory needed by the BGMV kernel exceeds the device limit";
-      return cudaErrorInvalidConfiguration;
-    }
-    if (!attr_set[dev]) {
-      err = cudaFuncSetAttribute(bgmv_coop_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_optin);
-      if (err != cudaSuccess) return err;
-      attr_set[dev] = true;
-    }
-  }
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bgmv_coop_kernel, kBgmvThreads,
-                                                      smem);
-  if (err != cudaSuccess) return err;
-  if (per_sm <= 0) {
-    *why = "the BGMV kernel does not fit on one SM";
-    return cudaErrorInvalidConfiguration;
-  }
-  const int units_max = items_max * kGroup;
-  const int grid = max(1, min(per_sm * sms, units_max));
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int* cnt = reinterpret_cast<int*>(ws);
-  int* done = cnt + items_max;
-  float* part = reinterpret_cast<float*>(ws + kCounterReserve);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cfg.gridDim = dim3((unsigned)grid, 1, 1);
-  cfg.blockDim = dim3(kBgmvThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  return cudaLaunchKernelEx(&cfg, bgmv_coop_kernel, p, cnt, done, part);
-}
 
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,
                         const char** why) {

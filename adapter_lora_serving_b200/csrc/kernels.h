@@ -126,16 +126,6 @@ inline void bgmv_pick_stages(int in, int S, int R, int* kb, int* nst) {
   }
 }
 
-// Bytes at the start of every workspace reserved for the per-item counters of
-// the cooperative BGMV kernel (zero between calls); other uses start after it.
-constexpr size_t kCounterReserve = 64 * 1024;
-
-// Workspace of the cooperative fused kernel: counters + partial h tiles.
-size_t bgmv_coop_workspace_bytes(int T, int slots, int R, int S);
-// Fused shrink + expand (apply_linear) in the BGMV regime, cooperative launch.
-cudaError_t bgmv_coop_launch(const BgmvParams& p, void* workspace, cudaStream_t stream,
-                             const char** why);
-
 // Launchers (bgmv.cu).  Return a cudaError_t from the launch.
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,
                         const char** why);

@@ -18,8 +18,7 @@
 // device memory.  Every call shares the one array, and it keeps what the last
 // call wrote: calls that may overlap on the GPU (different streams without an
 // ordering between them) race on it.  The kernels write every scratch value
-// they later read, and the per-item counters at its start are zero at load time
-// and are returned to zero by every call, so nothing needs clearing.
+// they later read, so nothing needs clearing between calls.
 #include <cuda_runtime.h>
 
 #include <cstdio>

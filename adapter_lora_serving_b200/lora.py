@@ -39,7 +39,7 @@ LORA_OP_GATHER_SHRINK = 3
 LORA_OP_APPLY_EMBEDDING = 4
 LORA_OP_EXPERT_APPLY = 5
 
-LORA_STATIC_SCRATCH_BYTES = 32 << 20
+LORA_STATIC_SCRATCH_BYTES = 16 << 20
 
 # (name, restype, argtypes) of every exported symbol.
 _P = ctypes.c_void_p

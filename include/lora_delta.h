@@ -127,13 +127,10 @@ LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const i
 
 /*
  * lora_apply_linear -- LoraBackend.apply_linear_ (shrink then expand, fused):
- * same arguments as lora_shrink + lora_expand; the partial h of the split
- * shrink goes through `workspace` (it stays in L2).  workspace must hold
- * lora_workspace_bytes(LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, regime)
- * bytes, be 16-byte aligned and be zero-filled before its first use: its first
- * 64 KiB hold per-item counters that every call leaves at zero again (after a
- * call that raised LORA_FLAG_TIMEOUT, zero it again).  Calls sharing one
- * workspace must not overlap on the GPU.
+ * same arguments as lora_shrink + lora_expand, with h kept on chip (BGMV) or in
+ * `workspace` (SGMV).  workspace must hold lora_workspace_bytes(
+ * LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, regime) bytes (may be NULL
+ * when that is 0).
  */
 LORA_API lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
                               const int32_t* ranks, const float* scalings,
@@ -201,7 +198,7 @@ LORA_API lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, con
  * delta (a plugin inside a runtime that owns all device memory and offers no
  * allocator, code running where cudaMalloc must not be called); this entry
  * point takes the lora_apply_linear arguments without the workspace and uses
- * a zero-initialised scratch array of LORA_STATIC_SCRATCH_BYTES compiled into the library
+ * a scratch array of LORA_STATIC_SCRATCH_BYTES compiled into the library
  * (every GPU that loads the library holds it until the process exits).
  * Shapes whose workspace (lora_workspace_bytes) exceeds that size return
  * LORA_ERR_UNSUPPORTED.  The first call on each device looks up the array's
@@ -210,7 +207,7 @@ LORA_API lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, con
  * the last call's contents (nothing needs clearing); calls that can overlap on
  * the GPU race on it.
  */
-#define LORA_STATIC_SCRATCH_BYTES (32u << 20)
+#define LORA_STATIC_SCRATCH_BYTES (16u << 20)
 LORA_API lora_status lora_apply_linear_noalloc(const void* x, void* y, const void* a, const void* b,
                                                const int32_t* ranks, const float* scalings,
                                                const int32_t* token_order,

@@ -67,7 +67,7 @@ class LinearDev:
                                           p.num_slices, regime)
         if ws_bytes and workspace is None:
             t = torch()
-            workspace = t.zeros(ws_bytes // 4 + 4, dtype=t.float32, device="cuda")
+            workspace = t.empty(ws_bytes // 4 + 4, dtype=t.float32, device="cuda")
         L.lora_apply_linear(self.x, self.y, self.a, self.b, self.ranks, self.scalings,
                             self.token_order, self.slot_indptr, p.T, p.n_in, p.slots, p.R,
                             out_slices or p.out_slices, regime=regime, workspace=workspace,

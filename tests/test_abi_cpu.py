@@ -113,10 +113,6 @@ def test_status_strings(lib):
 def test_host_queries(lib):
     assert L.lora_plan_tile(L.LORA_OP_APPLY_LINEAR, L.LORA_REGIME_BGMV) == 32
     assert L.lora_plan_tile(L.LORA_OP_EXPERT_APPLY, L.LORA_REGIME_AUTO) == 32
-    # 64 KiB of item counters + one partial h tile (32 tokens x S*roundup(R,16) fp32)
-    # per (item, k-split); items <= slots + ceil(T/32), 8 splits
-    items = 32 + 256 // 32
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
-                                  L.LORA_REGIME_BGMV) == 65536 + items * 8 * 32 * 48 * 4
-    assert L.lora_workspace_bytes(L.LORA_OP_SHRINK, 256, 32, 16, 3, L.LORA_REGIME_BGMV) == 0
+                                  L.LORA_REGIME_BGMV) == 0
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == L.LORA_REGIME_BGMV
