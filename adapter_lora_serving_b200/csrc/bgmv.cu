@@ -23,6 +23,8 @@
 
 namespace lora {
 
+static_assert(kTT == 32, "token masks are warp ballots: one token per lane of warp 0");
+
 namespace {
 
 struct Smem {
@@ -88,15 +90,25 @@ LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   const int cpr = min(p.kb, G.k1 - kbase) >> 3;   // 16-byte chunks per row
   const int Rpad = round_up_i(p.R, 16);
   const uint32_t stage = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
+  // (slice, rank row) of this warp's first A row, advanced by kBgmvThreads/32
+  // rows per step without a division per row
+  int ai = 0, ar = row_lo + warp;
+  if (row_lo + warp < G.nrows_a) {
+    ai = ar / rank;
+    ar -= ai * rank;
+  }
   for (int row = row_lo + warp; row < row_hi; row += kBgmvThreads / 32) {
     const __nv_bfloat16* src;
     uint32_t dst;
     if (row < G.nrows_a) {
-      const int i = row / rank;
-      const int r = row - i * rank;
       src = reinterpret_cast<const __nv_bfloat16*>(p.a) +
-            ((size_t)w * p.S * p.R + i * p.R + r) * p.in + kbase;
-      dst = stage + (uint32_t)((i * Rpad + r) * L.row_stride);
+            ((size_t)w * p.S * p.R + ai * p.R + ar) * p.in + kbase;
+      dst = stage + (uint32_t)((ai * Rpad + ar) * L.row_stride);
+      ar += kBgmvThreads / 32;
+      while (ar >= rank) {
+        ar -= rank;
+        ++ai;
+      }
     } else {
       const int t = row - G.nrows_a;
       const int tk = sm.tok[t];
@@ -210,7 +222,8 @@ LORA_DEV void produce_h(const BgmvParams& p, const BgmvLayout& L, const Smem& sm
   const int Rpad = round_up_i(p.R, 16);
   const int q4 = ceil_div_i(rank, 16) * 4;     // groups of 4 columns per slice
   const int per_t = p.S * q4;
-  const int total = kTT * per_t;
+  // rows of the token tiles the expand reads (8 * ceil(n / 8) <= kTT)
+  const int total = round_up_i(n, 8) * per_t;
   for (int e = threadIdx.x; e < total; e += kBgmvThreads) {
     const int t = e / per_t;
     const int q = e - t * per_t;
@@ -293,7 +306,7 @@ LORA_DEV void expand_mma(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   const int c = lane & 3;
   const int out = p.out;
   const int R = p.R;
-  const int ochunk = round_up_i(ceil_div_i(out, kGroup), 16);
+  const int ochunk = bgmv_ochunk(out);
   const int j0 = min(out, (int)crank * ochunk);
   const int j1 = min(out, j0 + ochunk);
   const int mtiles = ceil_div_i(j1 - j0, 16);
@@ -411,19 +424,279 @@ LORA_DEV void expand_mma(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   }
 }
 
+// The expand operands of one item, staged in the ring once the shrink no
+// longer needs it: this CTA's B columns [j0, j1) of adapter w as stored
+// ([cols][R] bf16) at the ring's start, then the y row of every live token of
+// the item over the same columns (row stride ystride bytes).
+struct ExStage {
+  uint8_t* bs;
+  uint8_t* ys;
+  int ystride;
+};
+
+LORA_DEV ExStage ex_stage_carve(const Smem& sm, const BgmvParams& p) {
+  const int oc = bgmv_ochunk(p.out);
+  ExStage X;
+  X.bs = sm.ring;
+  X.ys = sm.ring + round_up_i(oc * p.R * 2, 128);
+  X.ystride = oc * 2 + 16;
+  return X;
+}
+
+// Warp 0 issues the bulk copies of the staged operands of adapter w for the
+// live rows of the item; their bytes complete on bar.  Every address and size
+// is a multiple of 16 bytes: out, R and the slice edges are multiples of 8 and
+// j0 a multiple of 16.
+LORA_DEV void stage_expand(const BgmvParams& p, const Smem& sm, const ExStage& X, int w, int n,
+                           uint32_t rowmask, uint32_t crank, uint64_t* bar) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  const int oc = bgmv_ochunk(p.out);
+  const int j0 = min(p.out, (int)crank * oc);
+  const int cols = min(p.out, j0 + oc) - j0;
+  const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
+  const bool any = cols > 0 && live != 0u;
+  const uint32_t bbytes = (uint32_t)(cols * p.R * 2);
+  const uint32_t rbytes = (uint32_t)(cols * 2);
+  if (lane == 0) {
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, any ? bbytes + (uint32_t)__popc(live) * rbytes : 0u);
+  }
+  __syncwarp();
+  if (!any) return;
+  if (lane == 0)
+    bulk_g2s(X.bs, reinterpret_cast<const uint16_t*>(p.b) + ((size_t)w * p.out + j0) * p.R,
+             bbytes, bar);
+  if ((live >> lane) & 1u)
+    bulk_g2s(X.ys + lane * X.ystride,
+             reinterpret_cast<const uint16_t*>(p.y) + (size_t)sm.tok[lane] * p.out + j0, rbytes,
+             bar);
+}
+
+// L2 prefetch of what stage_expand will copy (issued when the item starts, so
+// the copies after the shrink find their bytes in L2).
+LORA_DEV void prefetch_expand(const BgmvParams& p, const Smem& sm, int w, int n, uint32_t rowmask,
+                              uint32_t crank) {
+  const int lane = threadIdx.x & 31;
+  const int oc = bgmv_ochunk(p.out);
+  const int j0 = min(p.out, (int)crank * oc);
+  const int cols = min(p.out, j0 + oc) - j0;
+  const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
+  if (cols <= 0 || live == 0u) return;
+  if (lane == 0)
+    bulk_prefetch_l2(reinterpret_cast<const uint16_t*>(p.b) + ((size_t)w * p.out + j0) * p.R,
+                     (uint32_t)(cols * p.R * 2));
+  if ((live >> lane) & 1u)
+    bulk_prefetch_l2(reinterpret_cast<const uint16_t*>(p.y) + (size_t)sm.tok[lane] * p.out + j0,
+                     (uint32_t)(cols * 2));
+}
+
+// Zero masks of the bf16 B elements k0..k0+3 at or past the rank (as
+// mask_rank4): .x covers (k0, k0+1), .y covers (k0+2, k0+3).
+LORA_DEV uint2 rank_mask4(int k0, int rank) {
+  return make_uint2((k0 < rank ? 0xffffu : 0u) | (k0 + 1 < rank ? 0xffff0000u : 0u),
+                    (k0 + 2 < rank ? 0xffffu : 0u) | (k0 + 3 < rank ? 0xffff0000u : 0u));
+}
+
+// Expand of a staged item with the m16n8k16 MMAs of expand_mma (same operands,
+// same order, so the same results): D[16 columns, 8 tokens] = B H^T per 16-column
+// tile of one slice, H = hi + lo.  B comes from the staged copy and y = bf16_rne(
+// y + scal * D) is written in place into the staged y rows (write_back_staged
+// stores them).  Per slice the h fragments of every token tile (one k-step) or
+// of the current one are held in registers, so a tile costs two B loads, two
+// MMAs per token tile and the y updates.  A 16-column tile may reach past the
+// end of its slice (slice edges are multiples of 8); those lanes are masked and
+// the next slice computes their columns.
+template <bool kOneStep>
+LORA_DEV void expand_staged_t(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                              const ExStage& X, int rank, float scal, int n, uint32_t rowmask,
+                              uint32_t crank) {
+  constexpr int kNT = kTT / 8;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int g = lane >> 2;
+  const int c = lane & 3;
+  const int R = p.R;
+  const int oc = bgmv_ochunk(p.out);
+  const int j0 = min(p.out, (int)crank * oc);
+  const int j1 = min(p.out, j0 + oc);
+  const int ksteps = ceil_div_i(rank, 16);
+  const int ntn = ceil_div_i(n, 8);
+  const uint16_t* bs = reinterpret_cast<const uint16_t*>(X.bs);
+  // live y rows of the item; this lane updates tokens 2c + e of each tile,
+  // whose rows start at (8 nt + 2c + e) * ystride in the staged copy
+  const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
+  uint8_t* ylane = X.ys + 2 * c * X.ystride;
+  const uint2 m0 = rank_mask4(4 * c, rank);
+
+#pragma unroll 1
+  for (int i = 0; i < p.S; ++i) {
+    const int ls0 = max(j0, p.slice_off[i]) - j0;
+    const int ls1 = min(j1, p.slice_off[i + 1]) - j0;
+    if (ls0 >= ls1) continue;
+    uint2 hh[kNT], hl[kNT];
+    if (kOneStep) {
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        if (nt < ntn) {
+          const int ho = (i * kTT + nt * 8 + g) * L.hst + 4 * c;
+          hh[nt] = *reinterpret_cast<const uint2*>(sm.hhi + ho);
+          hl[nt] = *reinterpret_cast<const uint2*>(sm.hlo + ho);
+        }
+      }
+    }
+#pragma unroll 1
+    for (int jt = ls0 + warp * 16; jt < ls1; jt += kBgmvThreads / 2) {
+      const int jl = jt + 2 * g;      // this lane's column pair, local to the chunk
+      const bool ok = jl < ls1;
+      float d[kNT][4];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) d[nt][k] = 0.f;
+      if (kOneStep) {
+        uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
+        if (ok) {
+          b0 = *reinterpret_cast<const uint2*>(bs + (size_t)jl * R + 4 * c);
+          b1 = *reinterpret_cast<const uint2*>(bs + (size_t)(jl + 1) * R + 4 * c);
+        }
+        b0 = make_uint2(b0.x & m0.x, b0.y & m0.y);
+        b1 = make_uint2(b1.x & m0.x, b1.y & m0.y);
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          if (nt < ntn) {
+            mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, hh[nt].x, hh[nt].y);
+            mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, hl[nt].x, hl[nt].y);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const int k0 = ks * 16 + 4 * c;
+          uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
+          if (ok && k0 < R) {
+            b0 = *reinterpret_cast<const uint2*>(bs + (size_t)jl * R + k0);
+            b1 = *reinterpret_cast<const uint2*>(bs + (size_t)(jl + 1) * R + k0);
+          }
+          const uint2 mk = rank_mask4(k0, rank);
+          b0 = make_uint2(b0.x & mk.x, b0.y & mk.y);
+          b1 = make_uint2(b1.x & mk.x, b1.y & mk.y);
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            if (nt < ntn) {
+              const int ho = (i * kTT + nt * 8 + g) * L.hst + k0;
+              const uint2 h1 = *reinterpret_cast<const uint2*>(sm.hhi + ho);
+              const uint2 h2 = *reinterpret_cast<const uint2*>(sm.hlo + ho);
+              mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, h1.x, h1.y);
+              mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, h2.x, h2.y);
+            }
+          }
+        }
+      }
+      if (ok) {
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          if (nt < ntn) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              if ((live >> (nt * 8 + 2 * c + e)) & 1u) {
+                uint32_t* yp = reinterpret_cast<uint32_t*>(
+                    ylane + (nt * 8 + e) * X.ystride + jl * 2);
+                const uint32_t yo = *yp;
+                *yp = pack_bf16x2(fmaf(scal, d[nt][e], bf16_lo(yo)),
+                                  fmaf(scal, d[nt][2 + e], bf16_hi(yo)));
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+LORA_DEV void expand_staged(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                            const ExStage& X, int rank, float scal, int n, uint32_t rowmask,
+                            uint32_t crank) {
+  if (rank <= 16)
+    expand_staged_t<true>(p, L, sm, X, rank, scal, n, rowmask, crank);
+  else
+    expand_staged_t<false>(p, L, sm, X, rank, scal, n, rowmask, crank);
+}
+
+// Stores the updated staged y rows of the live tokens (warp 0, one bulk copy
+// per row) and waits until the copies have read shared memory, so the ring can
+// be reused.  Every thread must call it after its expand_staged: the generic
+// writes are fenced towards the bulk copies and a block barrier orders them.
+LORA_DEV void write_back_staged(const BgmvParams& p, const Smem& sm, const ExStage& X, int n,
+                                uint32_t rowmask, uint32_t crank) {
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  const int oc = bgmv_ochunk(p.out);
+  const int j0 = min(p.out, (int)crank * oc);
+  const int cols = min(p.out, j0 + oc) - j0;
+  const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
+  if (cols > 0 && ((live >> lane) & 1u)) {
+    bulk_s2g(reinterpret_cast<uint16_t*>(p.y) + (size_t)sm.tok[lane] * p.out + j0,
+             X.ys + lane * X.ystride, (uint32_t)(cols * 2));
+    bulk_commit();
+    bulk_wait_read_all();
+  }
+  __syncwarp();
+}
+
+// Waits (bounded, warp-uniform) for the staged expand operands.
+LORA_DEV bool wait_staged(uint64_t* bar, uint32_t parity) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Expand of a staged item.  If the copies do not land within the wait limit
+// the warp raises LORA_FLAG_TIMEOUT, skips its columns and waits once more
+// (bounded) so that no copy is still writing the ring when it is reused; the
+// rows are then not stored.  Every thread of the CTA must call it.
+LORA_DEV void expand_after_stage(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                                 const ExStage& X, uint64_t* bar, uint32_t parity, int rank,
+                                 float scal, int n, uint32_t rowmask, uint32_t crank) {
+  const bool ok = wait_staged(bar, parity);
+  if (ok) {
+    expand_staged(p, L, sm, X, rank, scal, n, rowmask, crank);
+  } else {
+    if ((threadIdx.x & 31) == 0) raise_flag(p.flags, LORA_FLAG_TIMEOUT);
+    wait_staged(bar, parity);
+  }
+  // the rows are stored only when every warp saw its copies land
+  if (__syncthreads_or(ok ? 0 : 1) == 0) {
+    write_back_staged(p, sm, X, n, rowmask, crank);
+  }
+}
+
 }  // namespace
 
 template <int MODE>
-__global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) {
+__global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams p) {
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
   constexpr bool kScaled = (MODE == kModeFused || MODE == kModeExpand || MODE == kModeEmbed ||
                             MODE == kModeExpert);
   constexpr bool kExpands = kScaled;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int npref = (MODE == kModeExpert) ? p.num_experts : p.slots;
-  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst);
+  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst,
+                                   p.ex_stage ? bgmv_ex_stage_bytes(p.out, p.R) : 0);
   const Smem sm = carve(smem_raw, L);
   const int tid = threadIdx.x;
+  // Staged expand: B and y of an item are bulk-copied into the idle ring while
+  // the cluster reduces h; ebar counts their bytes (one phase per use).
+  const bool staged = kExpands && kClustered && p.ex_stage != 0;
+  uint64_t* ebar = reinterpret_cast<uint64_t*>(smem_raw);
+  const ExStage X = ex_stage_carve(sm, p);
+  uint32_t ephase = 0;
+  if (staged && tid == 0) {
+    mbar_init(ebar, 1);
+    fence_mbar_init();
+  }
 
   uint32_t crank, group, ngroups;
   if (kClustered) {
@@ -436,6 +709,19 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
     ngroups = gridDim.x / kGroup;
   }
 
+  // token_order of the first kTokCache positions, loaded while the planner's
+  // reads are in flight and kept in shared memory (the expert mode uses that
+  // region for its sub-batches instead).
+  constexpr int kTokCache = kTT * kTT;
+  constexpr int kTokPerThread = kTokCache / kBgmvThreads;
+  const int tokc_n = (MODE != kModeExpert) ? min(p.T, kTokCache) : 0;
+  int tv[kTokPerThread];
+#pragma unroll
+  for (int q = 0; q < kTokPerThread; ++q) {
+    const int i = tid + q * kBgmvThreads;
+    tv[q] = i < tokc_n ? p.token_order[i] : -1;
+  }
+
   const bool report = (blockIdx.x == 0);
   int total;
   if (MODE == kModeExpert) {
@@ -446,12 +732,19 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
                                       p.slots, p.T, p.R, kTT, sm.prefix, sm.scratch, p.flags,
                                       report);
   }
+#pragma unroll
+  for (int q = 0; q < kTokPerThread; ++q) {
+    const int i = tid + q * kBgmvThreads;
+    if (i < tokc_n) sm.sub_rows[i] = tv[q];
+  }
   if (kClustered) {
     // Trip counts of loops holding a cluster barrier come from rank 0, so every
     // CTA of a cluster takes the same barriers.
     if (tid == 0) sm.ctrl[0] = total;
     cluster_sync();
     total = dsmem_ld_s32(dsmem_addr(&sm.ctrl[0], 0));
+  } else {
+    __syncthreads();
   }
 
   int hpar = 0;
@@ -467,7 +760,8 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
       const float scal = kScaled ? p.scalings[s] : 0.f;
       const bool emb = (MODE == kModeEmbed || MODE == kModeGather);
       int t = -1;
-      if (tid < n && p0 + tid >= 0 && p0 + tid < p.T) t = p.token_order[p0 + tid];
+      if (tid < n && p0 + tid >= 0 && p0 + tid < p.T)
+        t = (p0 + tid < tokc_n) ? sm.sub_rows[p0 + tid] : p.token_order[p0 + tid];
       ShrinkGeom G = {};
       if (kClustered) {
         // the A rows do not depend on the tokens: start them while the reads land
@@ -488,18 +782,22 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
         }
         sm.tok[tid] = t;
         sm.ids[tid] = id;
+        const uint32_t tm = __ballot_sync(0xffffffffu, t >= 0);
+        const uint32_t im = __ballot_sync(0xffffffffu, id >= 0);
+        if (tid == 0) {
+          sm.ctrl[4 + 2 * (iter & 1)] = tm;
+          sm.ctrl[5 + 2 * (iter & 1)] = im;
+        }
       }
       __syncthreads();
-      uint32_t tokmask = 0, idmask = 0;
-#pragma unroll
-      for (int t = 0; t < kTT; ++t) {
-        if (sm.tok[t] >= 0) tokmask |= 1u << t;
-        if (sm.ids[t] >= 0) idmask |= 1u << t;
-      }
+      const uint32_t tokmask = (uint32_t)sm.ctrl[4 + 2 * (iter & 1)];
+      const uint32_t idmask = (uint32_t)sm.ctrl[5 + 2 * (iter & 1)];
       const uint32_t rowmask = emb ? (tokmask & idmask) : tokmask;
+      if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, s, n, rowmask, crank);
       if (kClustered) {
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
         shrink_partial(p, L, sm, G, s, rank, n, hp);
+        if (staged) stage_expand(p, sm, X, s, n, rowmask, crank, ebar);
         cluster_sync();
         produce_h<kFromCluster>(p, L, sm, hp, s, rank, n, rowmask, kExpands,
                                 MODE == kModeShrink, crank);
@@ -511,7 +809,14 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
                                MODE == kModeGather, crank);
       }
       __syncthreads();
-      if (kExpands) expand_mma(p, L, sm, s, rank, scal, n, rowmask, crank);
+      if (kExpands) {
+        if (staged) {
+          expand_after_stage(p, L, sm, X, ebar, ephase, rank, scal, n, rowmask, crank);
+          ephase ^= 1u;
+        } else {
+          expand_mma(p, L, sm, s, rank, scal, n, rowmask, crank);
+        }
+      }
       __syncthreads();
     } else {
       // ---- MoE item: chunk of one expert's rows, split by slot ----
@@ -583,13 +888,20 @@ __global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(const BgmvParams p) 
         if (tid < kTT) sm.tok[tid] = (tid < n) ? sm.sub_rows[q * kTT + tid] : -1;
         __syncthreads();
         const uint32_t mask = (n >= 32) ? 0xffffffffu : ((1u << n) - 1u);
+        if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, w, n, mask, crank);
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
         shrink_partial(p, L, sm, G, w, rank, n, hp);
+        if (staged) stage_expand(p, sm, X, w, n, mask, crank, ebar);
         cluster_sync();
         produce_h<kFromCluster>(p, L, sm, hp, w, rank, n, mask, true, false, crank);
         hpar ^= 1;
         __syncthreads();
-        expand_mma(p, L, sm, w, rank, scal, n, mask, crank);
+        if (staged) {
+          expand_after_stage(p, L, sm, X, ebar, ephase, rank, scal, n, mask, crank);
+          ephase ^= 1u;
+        } else {
+          expand_mma(p, L, sm, w, rank, scal, n, mask, crank);
+        }
         __syncthreads();
       }
     }
@@ -620,7 +932,13 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
   bgmv_pick_stages(p.in, p.S, p.R, &p.kb, &p.nst);
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
   const int npref = (MODE == kModeExpert) ? p.num_experts : p.slots;
-  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst);
+  const BgmvLayout L0 = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst, 0);
+  const int ex_bytes = bgmv_ex_stage_bytes(p.out, p.R);
+  p.ex_stage = ((MODE == kModeFused || MODE == kModeExpert) &&
+                ex_bytes <= max(p.nst * L0.stage_bytes, kExStageMax))
+                   ? 1
+                   : 0;
+  const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst, p.ex_stage ? ex_bytes : 0);
   auto kern = bgmv_kernel<MODE>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);

@@ -108,6 +108,10 @@ LORA_DEV void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
                "r"(smem_u32(src)), "r"(bytes)
                : "memory");
 }
+// Hint: pull [src, src + bytes) into L2 (src and bytes multiples of 16).
+LORA_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 LORA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 LORA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 LORA_DEV void bulk_wait_read_all() {

@@ -23,6 +23,7 @@ constexpr int kMaxKB = 512;      // input features per pipeline stage (upper bou
 constexpr int kRingBudget = 120 * 1024;  // shared-memory bytes for the staging ring
 constexpr int kMaxCombosPerWarp = 8;  // (16-row tile, 8-token tile) pairs per warp
 constexpr int kMaxSRp = 128;     // num_slices * roundup(R, 16) limit of this regime
+constexpr int kExStageMax = 96 * 1024;  // largest staged expand the ring is grown for
 
 enum BgmvMode : int {
   kModeFused = 0,   // shrink + expand (apply_linear)
@@ -58,6 +59,7 @@ struct BgmvParams {
   int num_pairs;
   int kb;         // input features per stage (multiple of 8)
   int nst;        // stages in the ring (1 or 2)
+  int ex_stage;   // 1: the expand operands of an item fit the ring and are staged there
   int slice_off[LORA_MAX_SLICES + 1];
 };
 
@@ -78,6 +80,17 @@ struct BgmvLayout {
 __host__ __device__ inline int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ inline int round_up_i(int a, int b) { return ceil_div_i(a, b) * b; }
 
+// Output columns each CTA of a cluster expands (multiple of 16).
+__host__ __device__ inline int bgmv_ochunk(int out) { return round_up_i(ceil_div_i(out, kGroup), 16); }
+
+// Bytes of the ring that the staged expand operands of one item take: this
+// CTA's B columns ([cols][R] bf16) and kTT rows of y over them, each row
+// padded by 16 bytes.
+__host__ __device__ inline int bgmv_ex_stage_bytes(int out, int R) {
+  const int oc = bgmv_ochunk(out);
+  return round_up_i(oc * R * 2, 128) + kTT * (oc * 2 + 16);
+}
+
 // Misc shared region (ints): tok[kTT], id[kTT], ctrl[8], scratch[8],
 // sub_s[kTT], sub_p[kTT], sub_cnt[kTT], sub_rows[kTT*kTT].
 constexpr int kMiscInts = kTT + kTT + 8 + 8 + 3 * kTT + kTT * kTT;
@@ -85,8 +98,10 @@ constexpr int kMiscInts = kTT + kTT + 8 + 8 + 3 * kTT + kTT * kTT;
 // Input features each CTA of a cluster reduces over (multiple of 8).
 __host__ __device__ inline int bgmv_kchunk(int in) { return round_up_i(ceil_div_i(in, kGroup), 8); }
 
+// ring_min: bytes the ring must hold besides its stages (the staged expand
+// operands), 0 when the expand is not staged.
 __host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, int R, int kb,
-                                                  int nst) {
+                                                  int nst, int ring_min) {
   BgmvLayout L;
   L.srp = S * round_up_i(R, 16);
   L.row_stride = kb * 2 + 16;
@@ -98,7 +113,7 @@ __host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, in
   off += round_up_i(kMiscInts * 4, 128);
   L.ring_off = off;
   const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpert);
-  if (ring) off += nst * L.stage_bytes;
+  if (ring) off += round_up_i(max(nst * L.stage_bytes, ring_min), 128);
   L.hpart_off = off;
   if (ring) off += 2 * kTT * L.srp * 4;
   L.hst = round_up_i(R, 16) + 8;
