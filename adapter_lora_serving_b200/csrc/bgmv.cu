@@ -78,53 +78,83 @@ LORA_DEV ShrinkGeom shrink_geom(const BgmvParams& p, int rank, uint32_t crank) {
   return G;
 }
 
-// Issue 16-byte copies of staged rows [row_lo, row_hi) of stage kb into ring
-// slot st.  Rows below nrows_a are live A rows; the next kTT rows are the
-// item's x rows (rows of invalid tokens are skipped).  A warp copies a row.
+// Which staged rows of a stage an issue covers.
+enum RowSet : int { kRowsA = 1, kRowsX = 2, kRowsAll = 3 };
+
+// Warp 0 issues the bulk copies (the TMA engine) of stage kb into ring slot st:
+// the live A rows of adapter w (rows below nrows_a, at i*Rpad + r) and/or the
+// item's x rows (tokens t < n with a valid token, at srp + t), kv input
+// features each.  Their bytes complete on bar; kRowsA only raises the expected
+// bytes, the other sets also arrive (one arrival per phase).  Every address and
+// size is a multiple of 16 bytes (in and the stage offsets are multiples of 8).
 LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                         const ShrinkGeom& G, int w, int rank, int kb, int st, int row_lo,
-                         int row_hi) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+                         const ShrinkGeom& G, int w, int rank, int n, int kb, int st, int set,
+                         uint64_t* bar) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
   const int kbase = G.k0 + kb * p.kb;
-  const int cpr = min(p.kb, G.k1 - kbase) >> 3;   // 16-byte chunks per row
+  const uint32_t rbytes = (uint32_t)(min(p.kb, G.k1 - kbase) * 2);
   const int Rpad = round_up_i(p.R, 16);
-  const uint32_t stage = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
-  // (slice, rank row) of this warp's first A row, advanced by kBgmvThreads/32
-  // rows per step without a division per row
-  int ai = 0, ar = row_lo + warp;
-  if (row_lo + warp < G.nrows_a) {
-    ai = ar / rank;
-    ar -= ai * rank;
+  uint8_t* stage = sm.ring + st * L.stage_bytes;
+  const bool want_a = (set & kRowsA) != 0 && G.nrows_a > 0;
+  const bool want_x = (set & kRowsX) != 0;
+  const int t = lane;
+  const bool xrow = want_x && t < n && sm.tok[t] >= 0;
+  const uint32_t xmask = __ballot_sync(0xffffffffu, xrow);
+  if (lane == 0) {
+    fence_proxy_async_smem();
+    const uint32_t bytes =
+        ((want_a ? (uint32_t)G.nrows_a : 0u) + (uint32_t)__popc(xmask)) * rbytes;
+    if (set == kRowsA)
+      mbar_expect_tx(bar, bytes);
+    else
+      mbar_arrive_expect_tx(bar, bytes);
   }
-  for (int row = row_lo + warp; row < row_hi; row += kBgmvThreads / 32) {
-    const __nv_bfloat16* src;
-    uint32_t dst;
-    if (row < G.nrows_a) {
-      src = reinterpret_cast<const __nv_bfloat16*>(p.a) +
-            ((size_t)w * p.S * p.R + ai * p.R + ar) * p.in + kbase;
-      dst = stage + (uint32_t)((ai * Rpad + ar) * L.row_stride);
-      ar += kBgmvThreads / 32;
+  __syncwarp();
+  if (want_a) {
+    // (slice, rank row) of this lane's first A row, advanced 32 rows per step
+    int ai = lane / rank;
+    int ar = lane - ai * rank;
+    for (int row = lane; row < G.nrows_a; row += 32) {
+      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(p.a) +
+                                 ((size_t)w * p.S * p.R + ai * p.R + ar) * p.in + kbase;
+      bulk_g2s(stage + (ai * Rpad + ar) * L.row_stride, src, rbytes, bar);
+      ar += 32;
       while (ar >= rank) {
         ar -= rank;
         ++ai;
       }
-    } else {
-      const int t = row - G.nrows_a;
-      const int tk = sm.tok[t];
-      if (tk < 0) continue;
-      src = reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)tk * p.in + kbase;
-      dst = stage + (uint32_t)((L.srp + t) * L.row_stride);
     }
-    for (int c = lane; c < cpr; c += 32) cp_async16(dst + c * 16, src + c * 8);
   }
+  if (xrow) {
+    const __nv_bfloat16* src =
+        reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)sm.tok[t] * p.in + kbase;
+    bulk_g2s(stage + (L.srp + t) * L.row_stride, src, rbytes, bar);
+  }
+}
+
+// Warp-uniform bounded wait for phase `parity` of bar; on timeout raises
+// LORA_FLAG_TIMEOUT and waits once more (bounded) so that no copy is still in
+// flight when the shared memory is reused.  Returns false on timeout.
+LORA_DEV bool wait_stage(uint64_t* bar, uint32_t parity, uint32_t* flags) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    ok = mbar_wait(bar, parity);
+    if (!ok) {
+      raise_flag(flags, LORA_FLAG_TIMEOUT);
+      mbar_wait(bar, parity);
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // MMAs of the shrink over this CTA's input features into hpart[t * srp +
 // i*Rpad + r] (every 16-row tile holding a live row, t < 8*ceil(n/8)).  The
-// caller has issued the A rows of stage 0 (uncommitted); this issues the rest.
+// caller has issued the A rows of stage 0 (kRowsA on sbar[0]); this issues the
+// rest.  sph holds the phase parity of each ring slot's barrier (bit st).
 LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                             const ShrinkGeom& G, int w, int rank, int n, float* hpart) {
+                             const ShrinkGeom& G, int w, int rank, int n, float* hpart,
+                             uint64_t* sbar, uint32_t& sph) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -142,17 +172,13 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
     for (int q = 0; q < 4; ++q) acc[c][q] = 0.f;
 
   if (G.nkb > 0) {
-    issue_rows(p, L, sm, G, w, rank, 0, 0, G.nrows_a, G.nrows_a + n);
-    cp_async_commit();
-    if (G.nkb > 1 && p.nst == 2) {
-      issue_rows(p, L, sm, G, w, rank, 1, 1, 0, G.nrows_a + n);
-      cp_async_commit();
-    }
+    issue_rows(p, L, sm, G, w, rank, n, 0, 0, kRowsX, &sbar[0]);
+    if (G.nkb > 1 && p.nst == 2) issue_rows(p, L, sm, G, w, rank, n, 1, 1, kRowsAll, &sbar[1]);
   }
   for (int kb = 0; kb < G.nkb; ++kb) {
     const int st = kb % p.nst;
-    if (kb + 1 < G.nkb && p.nst == 2) cp_async_wait<1>(); else cp_async_wait<0>();
-    __syncthreads();
+    wait_stage(&sbar[st], (sph >> st) & 1u, p.flags);
+    sph ^= 1u << st;
     const int kv = min(p.kb, G.k1 - (G.k0 + kb * p.kb));
     const int nks = ceil_div_i(kv, 16);
     const uint32_t stage_addr = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
@@ -182,10 +208,8 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
       }
     }
     __syncthreads();
-    if (kb + p.nst < G.nkb) {
-      issue_rows(p, L, sm, G, w, rank, kb + p.nst, st, 0, G.nrows_a + n);
-      cp_async_commit();
-    }
+    if (kb + p.nst < G.nkb)
+      issue_rows(p, L, sm, G, w, rank, n, kb + p.nst, st, kRowsAll, &sbar[st]);
   }
 
   const int g8 = lane >> 2;
@@ -498,30 +522,105 @@ LORA_DEV uint2 rank_mask4(int k0, int rank) {
                     (k0 + 2 < rank ? 0xffffu : 0u) | (k0 + 3 < rank ? 0xffff0000u : 0u));
 }
 
+constexpr int kExGroup = 4;   // 16-column tiles a warp expands per step
+
+// One step of the staged expand: kExGroup 16-column tiles (columns jt + 128 q)
+// of one slice and one 8-token tile.  All shared-memory loads of the step are
+// issued before any MMA or store (the B copy, the h tiles and the y rows do
+// not overlap), so the tiles' latencies overlap.  ks0 < ksteps k-steps of 16
+// ranks; hh/hl are the h fragments of k-step 0 when kOneStep.
+template <bool kOneStep>
+LORA_DEV void expand_step(const uint16_t* __restrict__ bs, const uint16_t* __restrict__ hhi,
+                          const uint16_t* __restrict__ hlo, uint8_t* __restrict__ yt, int ystride,
+                          int R, int hrow, int ksteps, int rank, uint2 m0, uint2 hh, uint2 hl,
+                          int jt, int ls1, int g, int c, uint32_t lv, float scal) {
+  int jl[kExGroup];
+  bool ok[kExGroup];
+  float d[kExGroup][4];
+  uint32_t yo[kExGroup][2];
+#pragma unroll
+  for (int q = 0; q < kExGroup; ++q) {
+    jl[q] = jt + q * (kBgmvThreads / 2) + 2 * g;
+    ok[q] = jl[q] < ls1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) d[q][k] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      yo[q][e] = (ok[q] && ((lv >> e) & 1u))
+                     ? *reinterpret_cast<const uint32_t*>(yt + e * ystride + jl[q] * 2)
+                     : 0u;
+  }
+  if (kOneStep) {
+    uint2 b0[kExGroup], b1[kExGroup];
+#pragma unroll
+    for (int q = 0; q < kExGroup; ++q) {
+      b0[q] = b1[q] = make_uint2(0u, 0u);
+      if (ok[q]) {
+        b0[q] = *reinterpret_cast<const uint2*>(bs + (size_t)jl[q] * R + 4 * c);
+        b1[q] = *reinterpret_cast<const uint2*>(bs + (size_t)(jl[q] + 1) * R + 4 * c);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kExGroup; ++q) {
+      const uint2 x0 = make_uint2(b0[q].x & m0.x, b0[q].y & m0.y);
+      const uint2 x1 = make_uint2(b1[q].x & m0.x, b1[q].y & m0.y);
+      mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, hh.x, hh.y);
+      mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, hl.x, hl.y);
+    }
+  } else {
+#pragma unroll 1
+    for (int ks = 0; ks < ksteps; ++ks) {
+      const int k0 = ks * 16 + 4 * c;
+      const uint2 mk = rank_mask4(k0, rank);
+      const uint2 h1 = *reinterpret_cast<const uint2*>(hhi + hrow + k0);
+      const uint2 h2 = *reinterpret_cast<const uint2*>(hlo + hrow + k0);
+#pragma unroll
+      for (int q = 0; q < kExGroup; ++q) {
+        uint2 x0 = make_uint2(0u, 0u), x1 = make_uint2(0u, 0u);
+        if (ok[q] && k0 < R) {
+          x0 = *reinterpret_cast<const uint2*>(bs + (size_t)jl[q] * R + k0);
+          x1 = *reinterpret_cast<const uint2*>(bs + (size_t)(jl[q] + 1) * R + k0);
+        }
+        x0 = make_uint2(x0.x & mk.x, x0.y & mk.y);
+        x1 = make_uint2(x1.x & mk.x, x1.y & mk.y);
+        mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, h1.x, h1.y);
+        mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, h2.x, h2.y);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kExGroup; ++q) {
+    if (!ok[q]) continue;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      if ((lv >> e) & 1u)
+        *reinterpret_cast<uint32_t*>(yt + e * ystride + jl[q] * 2) =
+            pack_bf16x2(fmaf(scal, d[q][e], bf16_lo(yo[q][e])),
+                        fmaf(scal, d[q][2 + e], bf16_hi(yo[q][e])));
+    }
+  }
+}
+
 // Expand of a staged item with the m16n8k16 MMAs of expand_mma (same operands,
 // same order, so the same results): D[16 columns, 8 tokens] = B H^T per 16-column
 // tile of one slice, H = hi + lo.  B comes from the staged copy and y = bf16_rne(
 // y + scal * D) is written in place into the staged y rows (write_back_staged
-// stores them).  Per slice the h fragments of every token tile (one k-step) or
-// of the current one are held in registers, so a tile costs two B loads, two
-// MMAs per token tile and the y updates.  A 16-column tile may reach past the
-// end of its slice (slice edges are multiples of 8); those lanes are masked and
-// the next slice computes their columns.
-template <bool kOneStep>
-LORA_DEV void expand_staged_t(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                              const ExStage& X, int rank, float scal, int n, uint32_t rowmask,
-                              uint32_t crank) {
-  constexpr int kNT = kTT / 8;
+// stores them).  A 16-column tile may reach past the end of its slice (slice
+// edges are multiples of 8); those lanes are masked and the next slice
+// computes their columns.
+LORA_DEV void expand_staged(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                            const ExStage& X, int rank, float scal, int n, uint32_t rowmask,
+                            uint32_t crank) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int g = lane >> 2;
   const int c = lane & 3;
-  const int R = p.R;
   const int oc = bgmv_ochunk(p.out);
   const int j0 = min(p.out, (int)crank * oc);
   const int j1 = min(p.out, j0 + oc);
   const int ksteps = ceil_div_i(rank, 16);
   const int ntn = ceil_div_i(n, 8);
+  const bool one = ksteps <= 1;
   const uint16_t* bs = reinterpret_cast<const uint16_t*>(X.bs);
   // live y rows of the item; this lane updates tokens 2c + e of each tile,
   // whose rows start at (8 nt + 2c + e) * ystride in the staged copy
@@ -534,116 +633,49 @@ LORA_DEV void expand_staged_t(const BgmvParams& p, const BgmvLayout& L, const Sm
     const int ls0 = max(j0, p.slice_off[i]) - j0;
     const int ls1 = min(j1, p.slice_off[i + 1]) - j0;
     if (ls0 >= ls1) continue;
-    uint2 hh[kNT], hl[kNT];
-    if (kOneStep) {
-#pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) {
-        if (nt < ntn) {
-          const int ho = (i * kTT + nt * 8 + g) * L.hst + 4 * c;
-          hh[nt] = *reinterpret_cast<const uint2*>(sm.hhi + ho);
-          hl[nt] = *reinterpret_cast<const uint2*>(sm.hlo + ho);
-        }
-      }
-    }
 #pragma unroll 1
-    for (int jt = ls0 + warp * 16; jt < ls1; jt += kBgmvThreads / 2) {
-      const int jl = jt + 2 * g;      // this lane's column pair, local to the chunk
-      const bool ok = jl < ls1;
-      float d[kNT][4];
-#pragma unroll
-      for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) d[nt][k] = 0.f;
-      if (kOneStep) {
-        uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
-        if (ok) {
-          b0 = *reinterpret_cast<const uint2*>(bs + (size_t)jl * R + 4 * c);
-          b1 = *reinterpret_cast<const uint2*>(bs + (size_t)(jl + 1) * R + 4 * c);
-        }
-        b0 = make_uint2(b0.x & m0.x, b0.y & m0.y);
-        b1 = make_uint2(b1.x & m0.x, b1.y & m0.y);
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-          if (nt < ntn) {
-            mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, hh[nt].x, hh[nt].y);
-            mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, hl[nt].x, hl[nt].y);
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const int k0 = ks * 16 + 4 * c;
-          uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
-          if (ok && k0 < R) {
-            b0 = *reinterpret_cast<const uint2*>(bs + (size_t)jl * R + k0);
-            b1 = *reinterpret_cast<const uint2*>(bs + (size_t)(jl + 1) * R + k0);
-          }
-          const uint2 mk = rank_mask4(k0, rank);
-          b0 = make_uint2(b0.x & mk.x, b0.y & mk.y);
-          b1 = make_uint2(b1.x & mk.x, b1.y & mk.y);
-#pragma unroll
-          for (int nt = 0; nt < kNT; ++nt) {
-            if (nt < ntn) {
-              const int ho = (i * kTT + nt * 8 + g) * L.hst + k0;
-              const uint2 h1 = *reinterpret_cast<const uint2*>(sm.hhi + ho);
-              const uint2 h2 = *reinterpret_cast<const uint2*>(sm.hlo + ho);
-              mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, h1.x, h1.y);
-              mma_bf16_16816(d[nt], b0.x, b1.x, b0.y, b1.y, h2.x, h2.y);
-            }
-          }
-        }
+    for (int nt = 0; nt < ntn; ++nt) {
+      const int hrow = (i * kTT + nt * 8 + g) * L.hst;
+      uint2 hh = make_uint2(0u, 0u), hl = make_uint2(0u, 0u);
+      if (one) {
+        hh = *reinterpret_cast<const uint2*>(sm.hhi + hrow + 4 * c);
+        hl = *reinterpret_cast<const uint2*>(sm.hlo + hrow + 4 * c);
       }
-      if (ok) {
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-          if (nt < ntn) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              if ((live >> (nt * 8 + 2 * c + e)) & 1u) {
-                uint32_t* yp = reinterpret_cast<uint32_t*>(
-                    ylane + (nt * 8 + e) * X.ystride + jl * 2);
-                const uint32_t yo = *yp;
-                *yp = pack_bf16x2(fmaf(scal, d[nt][e], bf16_lo(yo)),
-                                  fmaf(scal, d[nt][2 + e], bf16_hi(yo)));
-              }
-            }
-          }
-        }
+      const uint32_t lv = live >> (nt * 8 + 2 * c);
+      uint8_t* yt = ylane + nt * 8 * X.ystride;
+#pragma unroll 1
+      for (int jt = ls0 + warp * 16; jt < ls1; jt += kExGroup * (kBgmvThreads / 2)) {
+        if (one)
+          expand_step<true>(bs, sm.hhi, sm.hlo, yt, X.ystride, p.R, hrow, ksteps, rank, m0, hh,
+                            hl, jt, ls1, g, c, lv, scal);
+        else
+          expand_step<false>(bs, sm.hhi, sm.hlo, yt, X.ystride, p.R, hrow, ksteps, rank, m0, hh,
+                             hl, jt, ls1, g, c, lv, scal);
       }
     }
   }
 }
 
-LORA_DEV void expand_staged(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                            const ExStage& X, int rank, float scal, int n, uint32_t rowmask,
-                            uint32_t crank) {
-  if (rank <= 16)
-    expand_staged_t<true>(p, L, sm, X, rank, scal, n, rowmask, crank);
-  else
-    expand_staged_t<false>(p, L, sm, X, rank, scal, n, rowmask, crank);
-}
-
-// Stores the updated staged y rows of the live tokens (warp 0, one bulk copy
-// per row) and waits until the copies have read shared memory, so the ring can
-// be reused.  Every thread must call it after its expand_staged: the generic
-// writes are fenced towards the bulk copies and a block barrier orders them.
+// Stores the updated staged y rows of the live tokens: warp w copies rows
+// w, w + 8, ... with 16-byte loads and stores (a warp instruction moves 512
+// contiguous bytes of a row).  Every thread must call it after its
+// expand_staged.
 LORA_DEV void write_back_staged(const BgmvParams& p, const Smem& sm, const ExStage& X, int n,
                                 uint32_t rowmask, uint32_t crank) {
-  fence_proxy_async_smem();
   __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int oc = bgmv_ochunk(p.out);
   const int j0 = min(p.out, (int)crank * oc);
-  const int cols = min(p.out, j0 + oc) - j0;
+  const int cpr = (min(p.out, j0 + oc) - j0) >> 3;   // 16-byte chunks per row
   const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
-  if (cols > 0 && ((live >> lane) & 1u)) {
-    bulk_s2g(reinterpret_cast<uint16_t*>(p.y) + (size_t)sm.tok[lane] * p.out + j0,
-             X.ys + lane * X.ystride, (uint32_t)(cols * 2));
-    bulk_commit();
-    bulk_wait_read_all();
+  for (int t = warp; t < n; t += kBgmvThreads / 32) {
+    if (!((live >> t) & 1u)) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(X.ys + t * X.ystride);
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.y) +
+                                          (size_t)sm.tok[t] * p.out + j0);
+    for (int ch = lane; ch < cpr; ch += 32) dst[ch] = src[ch];
   }
-  __syncwarp();
 }
 
 // Waits (bounded, warp-uniform) for the staged expand operands.
@@ -691,10 +723,15 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   // the cluster reduces h; ebar counts their bytes (one phase per use).
   const bool staged = kExpands && kClustered && p.ex_stage != 0;
   uint64_t* ebar = reinterpret_cast<uint64_t*>(smem_raw);
+  // Ring slots' barriers: the bulk copies of a shrink stage complete on them.
+  uint64_t* sbar = ebar + 1;
+  uint32_t sph = 0;
   const ExStage X = ex_stage_carve(sm, p);
   uint32_t ephase = 0;
-  if (staged && tid == 0) {
+  if (tid == 0 && (staged || kClustered)) {
     mbar_init(ebar, 1);
+    mbar_init(&sbar[0], 1);
+    mbar_init(&sbar[1], 1);
     fence_mbar_init();
   }
 
@@ -737,6 +774,25 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
     const int i = tid + q * kBgmvThreads;
     if (i < tokc_n) sm.sub_rows[i] = tv[q];
   }
+  if (MODE != kModeExpert) {
+    // Addressing of this CTA's first kItemCache items, written by the thread
+    // of their slot (its planner reads are still in L1), so that an item
+    // starts without a dependent global load.
+    for (int sl = tid; sl < p.slots; sl += kBgmvThreads) {
+      const int i0 = sm.prefix[sl], i1 = sm.prefix[sl + 1];
+      if (i1 <= i0) continue;
+      for (int k = 0; k < kItemCache; ++k) {
+        const int item = (int)group + k * (int)ngroups;
+        if (item < i0 || item >= i1 || item >= total) continue;
+        const int p0 = p.slot_indptr[sl] + (item - i0) * kTT;
+        sm.sub_s[k] = sl;
+        sm.sub_s[kItemCache + k] = p.ranks[sl];
+        sm.sub_p[k] = p0;
+        sm.sub_p[kItemCache + k] = kScaled ? __float_as_int(p.scalings[sl]) : 0;
+        sm.sub_cnt[k] = max(0, min(kTT, p.slot_indptr[sl + 1] - p0));
+      }
+    }
+  }
   if (kClustered) {
     // Trip counts of loops holding a cluster barrier come from rank 0, so every
     // CTA of a cluster takes the same barriers.
@@ -752,12 +808,21 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   for (int item = (int)group; item < total; item += (int)ngroups, ++iter) {
     if (MODE != kModeExpert) {
       // ---- linear / embedding item: (slot, tile of kTT positions) ----
-      const int s = find_segment(sm.prefix, p.slots, item);
-      const int j = item - sm.prefix[s];
-      const int p0 = p.slot_indptr[s] + j * kTT;
-      const int n = max(0, min(kTT, p.slot_indptr[s + 1] - p0));
-      const int rank = p.ranks[s];
-      const float scal = kScaled ? p.scalings[s] : 0.f;
+      int s, p0, n, rank;
+      float scal;
+      if (iter < kItemCache) {
+        s = sm.sub_s[iter];
+        rank = sm.sub_s[kItemCache + iter];
+        p0 = sm.sub_p[iter];
+        scal = __int_as_float(sm.sub_p[kItemCache + iter]);
+        n = sm.sub_cnt[iter];
+      } else {
+        s = find_segment(sm.prefix, p.slots, item);
+        p0 = p.slot_indptr[s] + (item - sm.prefix[s]) * kTT;
+        n = max(0, min(kTT, p.slot_indptr[s + 1] - p0));
+        rank = p.ranks[s];
+        scal = kScaled ? p.scalings[s] : 0.f;
+      }
       const bool emb = (MODE == kModeEmbed || MODE == kModeGather);
       int t = -1;
       if (tid < n && p0 + tid >= 0 && p0 + tid < p.T)
@@ -766,7 +831,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       if (kClustered) {
         // the A rows do not depend on the tokens: start them while the reads land
         G = shrink_geom(p, rank, crank);
-        if (G.nkb > 0) issue_rows(p, L, sm, G, s, rank, 0, 0, 0, G.nrows_a);
+        if (G.nkb > 0) issue_rows(p, L, sm, G, s, rank, 0, 0, 0, kRowsA, &sbar[0]);
       }
       if (tid < kTT) {
         int id = -1;
@@ -796,7 +861,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, s, n, rowmask, crank);
       if (kClustered) {
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
-        shrink_partial(p, L, sm, G, s, rank, n, hp);
+        shrink_partial(p, L, sm, G, s, rank, n, hp, sbar, sph);
         if (staged) stage_expand(p, sm, X, s, n, rowmask, crank, ebar);
         cluster_sync();
         produce_h<kFromCluster>(p, L, sm, hp, s, rank, n, rowmask, kExpands,
@@ -884,13 +949,13 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         const int rank = mine ? p.ranks[sl] : 0;
         const float scal = mine ? p.scalings[sl] : 0.f;
         const ShrinkGeom G = shrink_geom(p, rank, crank);
-        if (G.nkb > 0 && rank > 0) issue_rows(p, L, sm, G, w, rank, 0, 0, 0, G.nrows_a);
+        if (G.nkb > 0 && rank > 0) issue_rows(p, L, sm, G, w, rank, 0, 0, 0, kRowsA, &sbar[0]);
         if (tid < kTT) sm.tok[tid] = (tid < n) ? sm.sub_rows[q * kTT + tid] : -1;
         __syncthreads();
         const uint32_t mask = (n >= 32) ? 0xffffffffu : ((1u << n) - 1u);
         if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, w, n, mask, crank);
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
-        shrink_partial(p, L, sm, G, w, rank, n, hp);
+        shrink_partial(p, L, sm, G, w, rank, n, hp, sbar, sph);
         if (staged) stage_expand(p, sm, X, w, n, mask, crank, ebar);
         cluster_sync();
         produce_h<kFromCluster>(p, L, sm, hp, w, rank, n, mask, true, false, crank);

@@ -21,8 +21,11 @@ constexpr int kTT = 32;          // tokens (sorted rows) per work item
 constexpr int kGroup = 8;        // CTAs per work item (cluster size)
 constexpr int kMaxKB = 512;      // input features per pipeline stage (upper bound)
 constexpr int kRingBudget = 120 * 1024;  // shared-memory bytes for the staging ring
-constexpr int kMaxCombosPerWarp = 8;  // (16-row tile, 8-token tile) pairs per warp
+constexpr int kMaxCombosPerWarp = 4;  // (16-row tile, 8-token tile) pairs per warp:
+                                      // (kMaxSRp/16) * (kTT/8) / 8 warps
 constexpr int kMaxSRp = 128;     // num_slices * roundup(R, 16) limit of this regime
+static_assert((kMaxSRp / 16) * (kTT / 8) <= kMaxCombosPerWarp * (kBgmvThreads / 32),
+              "every (row tile, token tile) pair of the shrink has a warp slot");
 constexpr int kExStageMax = 96 * 1024;  // largest staged expand the ring is grown for
 
 enum BgmvMode : int {
@@ -90,6 +93,10 @@ __host__ __device__ inline int bgmv_ex_stage_bytes(int out, int R) {
   const int oc = bgmv_ochunk(out);
   return round_up_i(oc * R * 2, 128) + kTT * (oc * 2 + 16);
 }
+
+// Items per CTA whose addressing the planner caches in shared memory (linear
+// modes, in the sub-batch arrays the expert mode uses otherwise).
+constexpr int kItemCache = 8;
 
 // Misc shared region (ints): tok[kTT], id[kTT], ctrl[8], scratch[8],
 // sub_s[kTT], sub_p[kTT], sub_cnt[kTT], sub_rows[kTT*kTT].
