@@ -12,7 +12,8 @@
 //         coalesced row writes.
 // Both kernels are persistent (one CTA per SM over a contiguous run of work
 // units) and warp-specialised: warp 0 loads, warp 1 issues MMAs (one thread),
-// warps 2-5 drain TMEM.  Every wait is bounded; on timeout the CTA raises
+// the other warps drain TMEM (shrink: 4; expand: 16, each 32 rows x 32
+// columns).  Every wait is bounded; on timeout the CTA raises
 // LORA_FLAG_TIMEOUT, stops, frees its TMEM and exits.
 //
 // Sources: mstar.engine.resources.lora.backend (LoraBackend.shrink,
@@ -31,7 +32,8 @@ namespace lora {
 namespace {
 
 constexpr int kSgThreads = 192;   // shrink: 6 warps
-constexpr int kExThreads = 320;   // expand: 10 warps (8 epilogue warps)
+constexpr int kExEpiWarps = 16;   // expand epilogue: 4 TMEM lane quarters x 4 column groups
+constexpr int kExThreads = 32 * (2 + kExEpiWarps);   // expand: producer, MMA, epilogue
 constexpr int kNY = 3;            // y staging buffers (prefetch two units ahead)
 constexpr int kTM = kSgmvTileM;   // 128 tokens per tile (MMA M)
 constexpr int kBN = 128;          // output columns per expand unit (MMA N)
@@ -173,9 +175,9 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 8);   // one arrival per epilogue warp
+      mbar_init(&accempty[i], kExEpiWarps);   // one arrival per epilogue warp
     }
-    mbar_init(hready, 256);   // one arrival per epilogue thread
+    mbar_init(hready, 32 * kExEpiWarps);   // one arrival per epilogue thread
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmap_b);
@@ -257,11 +259,11 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
       __syncwarp();
     }
   } else {
-    // ---------------- epilogue: warps 2..9 ----------------
+    // ---------------- epilogue: warps 2..17 ----------------
     // Warp w reads TMEM lanes 32*(w%4).. (one token row per thread) and owns
-    // half of the unit's 128 columns.
+    // the 32 columns [32 cg, 32 cg + 32) of the unit, cg = (w - 2) / 4.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int cg = (warp - 2) >> 2;
     const int m = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(p.y);
@@ -273,17 +275,17 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
       const int t = p.token_order[V.p0 + m];
       return (t >= 0 && t < p.T) ? t : -1;
     };
-    // The warp's 32 rows x 64 columns of y, as 16-byte copies: lane l takes
-    // chunk l % 8 of row 4j + l / 8, so an instruction moves four full
-    // 128-byte row segments.  `t` is this lane's own row token; rows read
-    // their token from the lane that owns them.
+    // The warp's 32 rows x 32 columns of y, as 16-byte copies: lane l takes
+    // chunk l % 4 of row 8j + l / 4, so an instruction moves eight 64-byte row
+    // segments.  `t` is this lane's own row token; rows read their token from
+    // the lane that owns them.
     auto prefetch_y = [&](const UnitCursor& V, int t, int buf) {
-      const int c = half * 8 + (lane & 7);
+      const int c = cg * 4 + (lane & 3);
       const bool cok = c < (V.width >> 3);
       const uint32_t base_s = smem_u32(ystage) + (uint32_t)(buf * kTM + quarter * 32) * kYRow;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int r = 4 * j + (lane >> 3);
+      for (int j = 0; j < 4; ++j) {
+        const int r = 8 * j + (lane >> 2);
         const int tr = __shfl_sync(0xffffffffu, t, r);
         if (tr >= 0 && cok)
           cp_async16(base_s + (uint32_t)r * kYRow + c * 16, yb + (size_t)tr * p.out + V.col0 + c * 8);
@@ -311,6 +313,11 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     } else {
       cp_async_commit();
     }
+    // per item: the slot's rank and scaling, this row's validity and id
+    int rank = 0;
+    float scal = 0.f;
+    bool row_ok = false;
+    int id = -1;
     for (int k = 0; k < nloc; ++k) {
       // keep two units of y in flight
       if (k + 2 < nloc) {
@@ -320,23 +327,24 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
         cp_async_commit();
       }
       const bool new_item = U.item != prev_item;
-      if (new_item && half == 0 && m < U.n && tok < 0 && U.col0 == 0)
-        raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
-      const int rank = p.ranks[U.s];
-      const float scal = p.scalings[U.s];
-      bool row_ok = tok >= 0;
-      int id = -1;
-      if (p.h == nullptr && row_ok) {
-        id = p.ids[tok];
-        if (id < 0 || id >= p.vocab) row_ok = false;
+      if (new_item) {
+        if (cg == 0 && m < U.n && tok < 0 && U.col0 == 0) raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
+        rank = p.ranks[U.s];
+        scal = p.scalings[U.s];
+        row_ok = tok >= 0;
+        id = -1;
+        if (p.h == nullptr && row_ok) {
+          id = p.ids[tok];
+          if (id < 0 || id >= p.vocab) row_ok = false;
+        }
       }
       if (new_item || U.slice != prev_slice) {
         // Build H (hi and lo) for (tile, slice); the MMAs of the previous unit
-        // are complete, since its epilogue waited for them.  The two warps of a
-        // row split its 16-byte chunks.
+        // are complete, since its epilogue waited for them.  The four warps of
+        // a row split its 16-byte chunks.
         const int Kp = ceil_div_i(rank, 16) * 16;
         const int i = U.slice;
-        for (int c8 = half * 8; c8 < Kp; c8 += 16) {
+        for (int c8 = cg * 8; c8 < Kp; c8 += 32) {
           float v[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -378,26 +386,23 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
       __syncwarp();   // the staged rows were copied by other lanes of this warp
       uint8_t* ybuf = ystage + (size_t)((k % kNY) * kTM) * kYRow;
       uint8_t* yrow = ybuf + (size_t)m * kYRow;
+      const int c0 = cg * 32;                   // first column of this warp
+      if (c0 < U.width) {                       // warp-uniform
+        float acc[32];
+        tmem_ld_32x32(tmem_base + lane_addr + (uint32_t)(as * kBN + c0), acc);
+        if (row_ok) {
 #pragma unroll
-      for (int cg = 0; cg < 2; ++cg) {
-        const int c0 = half * 64 + cg * 32;     // first column of this group
-        if (c0 < U.width) {                     // warp-uniform
-          float acc[32];
-          tmem_ld_32x32(tmem_base + lane_addr + (uint32_t)(as * kBN + c0), acc);
-          if (row_ok) {
+          for (int q = 0; q < 4; ++q) {
+            if (c0 + q * 8 < U.width) {
+              const uint4 yv = *reinterpret_cast<const uint4*>(yrow + c0 * 2 + q * 16);
+              uint32_t w[4] = {yv.x, yv.y, yv.z, yv.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (c0 + q * 8 < U.width) {
-                const uint4 yv = *reinterpret_cast<const uint4*>(yrow + c0 * 2 + q * 16);
-                uint32_t w[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int c = q * 8 + e * 2;
-                  w[e] = pack_bf16x2(fmaf(scal, acc[c], bf16_lo(w[e])),
-                                     fmaf(scal, acc[c + 1], bf16_hi(w[e])));
-                }
-                *reinterpret_cast<uint4*>(yrow + c0 * 2 + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int e = 0; e < 4; ++e) {
+                const int c = q * 8 + e * 2;
+                w[e] = pack_bf16x2(fmaf(scal, acc[c], bf16_lo(w[e])),
+                                   fmaf(scal, acc[c + 1], bf16_hi(w[e])));
               }
+              *reinterpret_cast<uint4*>(yrow + c0 * 2 + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
@@ -405,14 +410,14 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[as]);
-      // coalesced write-back of the warp's 32 rows x 64 columns
+      // coalesced write-back of the warp's 32 rows x 32 columns
       {
-        const int c = half * 8 + (lane & 7);
+        const int c = cg * 4 + (lane & 3);
         const bool cok = c < (U.width >> 3);
         const int tl = row_ok ? tok : -1;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int r = 4 * j + (lane >> 3);
+        for (int j = 0; j < 4; ++j) {
+          const int r = 8 * j + (lane >> 2);
           const int tr = __shfl_sync(0xffffffffu, tl, r);
           if (tr >= 0 && cok) {
             const uint4 v = *reinterpret_cast<const uint4*>(ybuf + (size_t)(quarter * 32 + r) * kYRow + c * 16);
