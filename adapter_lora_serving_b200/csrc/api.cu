@@ -399,8 +399,9 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
   p.S = num_slices; p.out = out; p.num_experts = num_experts; p.num_pairs = num_pairs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const char* why = nullptr;
+  // one CTA per work item (a chunk of one expert's rows)
   const int bound = linear_items_bound(rows_cap, num_experts, lora::kTT);
-  cudaError_t err = lora::bgmv_launch(lora::kModeExpert, p, bound, s, &why);
+  cudaError_t err = lora::bgmv_launch(lora::kModeExpertSolo, p, bound, s, &why);
   if (err != cudaSuccess) return cuda_fail(err, op, why);
   return ok();
 }

@@ -70,9 +70,8 @@ struct ShrinkGeom {
 
 LORA_DEV ShrinkGeom shrink_geom(const BgmvParams& p, int rank, uint32_t crank) {
   ShrinkGeom G;
-  const int kchunk = bgmv_kchunk(p.in);
-  G.k0 = min(p.in, (int)crank * kchunk);
-  G.k1 = min(p.in, G.k0 + kchunk);
+  G.k0 = min(p.in, (int)crank * p.kchunk);
+  G.k1 = min(p.in, G.k0 + p.kchunk);
   G.nkb = ceil_div_i(G.k1 - G.k0, p.kb);
   G.nrows_a = p.S * rank;
   return G;
@@ -232,7 +231,7 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
 }
 
 // Where the h of an item comes from.
-enum HSource : int { kFromCluster = 0, kFromGlobal = 1, kFromGather = 2 };
+enum HSource : int { kFromCluster = 0, kFromGlobal = 1, kFromGather = 2, kFromLocal = 3 };
 
 // Produce h for every (token t < kTT, slice i, column r < roundup16(rank)) of
 // the item -- the value for live tokens and r < rank, 0 elsewhere -- four
@@ -263,6 +262,9 @@ LORA_DEV void produce_h(const BgmvParams& p, const BgmvLayout& L, const Smem& sm
           const float4 f = dsmem_ld_f32x4(dsmem_addr(src, (uint32_t)c));
           v[0] += f.x; v[1] += f.y; v[2] += f.z; v[3] += f.w;
         }
+      } else if (SRC == kFromLocal) {
+        const float4 f = *reinterpret_cast<const float4*>(hpart + t * L.srp + i * Rpad + r0);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
       } else if (SRC == kFromGlobal) {
         const float* hg = p.h + (size_t)sm.tok[t] * p.S * p.R + i * p.R + r0;
 #pragma unroll
@@ -313,7 +315,7 @@ LORA_DEV uint2 mask_rank4(uint2 v, int k0, int rank) {
   return make_uint2(v.x & m0, v.y & m1);
 }
 
-// Expand of one item over this CTA's share of the output columns with
+// Expand of one item over the output columns [j0, j1) with
 // m16n8k16 MMAs: D[16 columns, 8 tokens] = B[16 columns, 16 ranks] H^T.
 // MMA row m < 8 is column 2m and row m + 8 is column 2m + 1 of the tile, and
 // MMA k (2c + e) / (2c + 8 + e) is rank 4c + e / 4c + 2 + e, so each lane
@@ -321,7 +323,7 @@ LORA_DEV uint2 mask_rank4(uint2 v, int k0, int rank) {
 // tokens.  H = hi + lo in bf16 (two MMAs, fp32 accumulate); then
 // y = bf16_rne(y + scal * D) on the live rows.
 LORA_DEV void expand_mma(const BgmvParams& p, const BgmvLayout& L, const Smem& sm, int w,
-                         int rank, float scal, int n, uint32_t rowmask, uint32_t crank) {
+                         int rank, float scal, int n, uint32_t rowmask, int j0, int j1) {
   constexpr int kMT = 3;              // 16-column tiles per warp per pass
   constexpr int kNT = kTT / 8;        // 8-token tiles
   const int lane = threadIdx.x & 31;
@@ -330,9 +332,6 @@ LORA_DEV void expand_mma(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   const int c = lane & 3;
   const int out = p.out;
   const int R = p.R;
-  const int ochunk = bgmv_ochunk(out);
-  const int j0 = min(out, (int)crank * ochunk);
-  const int j1 = min(out, j0 + ochunk);
   const int mtiles = ceil_div_i(j1 - j0, 16);
   const int ksteps = ceil_div_i(rank, 16);
   const int ntn = ceil_div_i(n, 8);
@@ -710,11 +709,12 @@ LORA_DEV void expand_after_stage(const BgmvParams& p, const BgmvLayout& L, const
 template <int MODE>
 __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams p) {
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
-  constexpr bool kScaled = (MODE == kModeFused || MODE == kModeExpand || MODE == kModeEmbed ||
-                            MODE == kModeExpert);
+  constexpr bool kSolo = (MODE == kModeExpertSolo);
+  constexpr bool kMoE = (MODE == kModeExpert || kSolo);
+  constexpr bool kScaled = (MODE == kModeFused || MODE == kModeExpand || MODE == kModeEmbed || kMoE);
   constexpr bool kExpands = kScaled;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  const int npref = (MODE == kModeExpert) ? p.num_experts : p.slots;
+  const int npref = kMoE ? p.num_experts : p.slots;
   const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst,
                                    p.ex_stage ? bgmv_ex_stage_bytes(p.out, p.R) : 0);
   const Smem sm = carve(smem_raw, L);
@@ -728,7 +728,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   uint32_t sph = 0;
   const ExStage X = ex_stage_carve(sm, p);
   uint32_t ephase = 0;
-  if (tid == 0 && (staged || kClustered)) {
+  if (tid == 0 && (staged || kClustered || kSolo)) {
     mbar_init(ebar, 1);
     mbar_init(&sbar[0], 1);
     mbar_init(&sbar[1], 1);
@@ -740,6 +740,10 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
     crank = cluster_ctarank();
     group = cluster_id_x();
     ngroups = num_clusters_x();
+  } else if (kSolo) {
+    crank = 0;
+    group = blockIdx.x;
+    ngroups = gridDim.x;
   } else {
     crank = blockIdx.x % kGroup;
     group = blockIdx.x / kGroup;
@@ -751,7 +755,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   // region for its sub-batches instead).
   constexpr int kTokCache = kTT * kTT;
   constexpr int kTokPerThread = kTokCache / kBgmvThreads;
-  const int tokc_n = (MODE != kModeExpert) ? min(p.T, kTokCache) : 0;
+  const int tokc_n = kMoE ? 0 : min(p.T, kTokCache);
   int tv[kTokPerThread];
 #pragma unroll
   for (int q = 0; q < kTokPerThread; ++q) {
@@ -761,7 +765,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
 
   const bool report = (blockIdx.x == 0);
   int total;
-  if (MODE == kModeExpert) {
+  if (kMoE) {
     total = plan_expert<kBgmvThreads>(p.expert_offsets, p.pair_index, p.num_experts, p.slots, p.T,
                                       kTT, sm.prefix, sm.scratch, p.flags, report);
   } else {
@@ -774,7 +778,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
     const int i = tid + q * kBgmvThreads;
     if (i < tokc_n) sm.sub_rows[i] = tv[q];
   }
-  if (MODE != kModeExpert) {
+  if (!kMoE) {
     // Addressing of this CTA's first kItemCache items, written by the thread
     // of their slot (its planner reads are still in L1), so that an item
     // starts without a dependent global load.
@@ -806,7 +810,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   int hpar = 0;
   int iter = 0;
   for (int item = (int)group; item < total; item += (int)ngroups, ++iter) {
-    if (MODE != kModeExpert) {
+    if (!kMoE) {
       // ---- linear / embedding item: (slot, tile of kTT positions) ----
       int s, p0, n, rank;
       float scal;
@@ -879,7 +883,9 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
           expand_after_stage(p, L, sm, X, ebar, ephase, rank, scal, n, rowmask, crank);
           ephase ^= 1u;
         } else {
-          expand_mma(p, L, sm, s, rank, scal, n, rowmask, crank);
+          const int oc = bgmv_ochunk(p.out);
+          const int j0 = min(p.out, (int)crank * oc);
+          expand_mma(p, L, sm, s, rank, scal, n, rowmask, j0, min(p.out, j0 + oc));
         }
       }
       __syncthreads();
@@ -891,56 +897,65 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       const int start = p.expert_offsets[e] + chunk * kTT;
       const int m = max(0, min(kTT, p.expert_offsets[e + 1] - start));
       int* nsub_slot = &sm.ctrl[2 + (iter & 1)];
-      if (tid == 0) {
+      if (tid < kTT) {
+        // lane q classifies row start + q (the fold's skip rules) ...
+        const int q = tid;
         uint32_t bad = 0;
-        int rs[kTT];
-        int rp[kTT];
-        for (int q = 0; q < kTT; ++q) {
-          rs[q] = -1;
-          rp[q] = -1;
-          if (q >= m) continue;
-          const int rho = start + q;
-          if (rho < 0 || rho >= p.T) continue;
+        int rs = 0x7fffffff, rp = -1;
+        const int rho = start + q;
+        if (q < m && rho >= 0 && rho < p.T) {
           const int sl = p.row_slot[rho];
-          if (sl == -1) continue;
-          if (sl < -1 || sl >= p.slots) { bad |= LORA_FLAG_BAD_SLOT; continue; }
-          const int pi = p.pair_index[(size_t)sl * E + e];
-          if (pi == -1) continue;
-          if (pi < -1 || pi >= p.num_pairs) { bad |= LORA_FLAG_BAD_PAIR; continue; }
-          const int r = p.ranks[sl];
-          if (r < 0 || r > p.R) { bad |= LORA_FLAG_BAD_RANK; continue; }
-          if (r == 0 || p.scalings[sl] == 0.0f) continue;
-          rs[q] = sl;
-          rp[q] = pi;
-        }
-        // sub-batches in ascending slot order, rows in row order
-        int nsub = 0;
-        int last = -1;
-        while (true) {
-          int best = 0x7fffffff;
-          for (int q = 0; q < kTT; ++q)
-            if (rs[q] > last && rs[q] < best) best = rs[q];
-          if (best == 0x7fffffff) break;
-          int cnt = 0;
-          for (int q = 0; q < kTT; ++q) {
-            if (rs[q] == best) {
-              sm.sub_rows[nsub * kTT + cnt] = start + q;
-              sm.sub_p[nsub] = rp[q];
-              ++cnt;
+          if (sl < -1 || sl >= p.slots) {
+            bad = LORA_FLAG_BAD_SLOT;
+          } else if (sl != -1) {
+            const int pi = p.pair_index[(size_t)sl * E + e];
+            if (pi != -1) {
+              if (pi < -1 || pi >= p.num_pairs) {
+                bad = LORA_FLAG_BAD_PAIR;
+              } else {
+                const int r = p.ranks[sl];
+                if (r < 0 || r > p.R) {
+                  bad = LORA_FLAG_BAD_RANK;
+                } else if (r != 0 && p.scalings[sl] != 0.0f) {
+                  rs = sl;
+                  rp = pi;
+                }
+              }
             }
           }
-          sm.sub_s[nsub] = best;
-          sm.sub_cnt[nsub] = cnt;
+        }
+        // ... and the warp forms the sub-batches: ascending slot order, rows in
+        // row order
+        const uint32_t lt = (1u << q) - 1u;
+        int nsub = 0;
+        for (int last = -1;;) {
+          const int best = (int)__reduce_min_sync(0xffffffffu, (unsigned)(rs > last ? rs : 0x7fffffff));
+          if (best == 0x7fffffff) break;
+          const uint32_t mk = __ballot_sync(0xffffffffu, rs == best);
+          if (rs == best) {
+            sm.sub_rows[nsub * kTT + __popc(mk & lt)] = rho;
+            if ((mk & lt) == 0u) {
+              sm.sub_p[nsub] = rp;
+              sm.sub_s[nsub] = best;
+              sm.sub_cnt[nsub] = __popc(mk);
+            }
+          }
           ++nsub;
           last = best;
         }
-        *nsub_slot = nsub;
-        if (crank == 0) raise_flag(p.flags, bad);
+        bad = __reduce_or_sync(0xffffffffu, bad);
+        if (q == 0) {
+          *nsub_slot = nsub;
+          if (crank == 0) raise_flag(p.flags, bad);
+        }
       }
       __syncthreads();
       const int my_nsub = *nsub_slot;
-      cluster_sync();
-      const int nsub = dsmem_ld_s32(dsmem_addr(nsub_slot, 0));
+      int nsub = my_nsub;
+      if (!kSolo) {
+        cluster_sync();
+        nsub = dsmem_ld_s32(dsmem_addr(nsub_slot, 0));
+      }
       for (int q = 0; q < nsub; ++q) {
         const bool mine = q < my_nsub;
         const int sl = mine ? sm.sub_s[q] : 0;
@@ -948,7 +963,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         const int n = mine ? sm.sub_cnt[q] : 0;
         const int rank = mine ? p.ranks[sl] : 0;
         const float scal = mine ? p.scalings[sl] : 0.f;
-        const ShrinkGeom G = shrink_geom(p, rank, crank);
+        const ShrinkGeom G = shrink_geom(p, rank, kSolo ? 0u : crank);
         if (G.nkb > 0 && rank > 0) issue_rows(p, L, sm, G, w, rank, 0, 0, 0, kRowsA, &sbar[0]);
         if (tid < kTT) sm.tok[tid] = (tid < n) ? sm.sub_rows[q * kTT + tid] : -1;
         __syncthreads();
@@ -956,16 +971,25 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, w, n, mask, crank);
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
         shrink_partial(p, L, sm, G, w, rank, n, hp, sbar, sph);
-        if (staged) stage_expand(p, sm, X, w, n, mask, crank, ebar);
-        cluster_sync();
-        produce_h<kFromCluster>(p, L, sm, hp, w, rank, n, mask, true, false, crank);
+        if (kSolo) {
+          __syncthreads();
+          produce_h<kFromLocal>(p, L, sm, hp, w, rank, n, mask, true, false, 0);
+        } else {
+          if (staged) stage_expand(p, sm, X, w, n, mask, crank, ebar);
+          cluster_sync();
+          produce_h<kFromCluster>(p, L, sm, hp, w, rank, n, mask, true, false, crank);
+        }
         hpar ^= 1;
         __syncthreads();
         if (staged) {
           expand_after_stage(p, L, sm, X, ebar, ephase, rank, scal, n, mask, crank);
           ephase ^= 1u;
+        } else if (kSolo) {
+          expand_mma(p, L, sm, w, rank, scal, n, mask, 0, p.out);
         } else {
-          expand_mma(p, L, sm, w, rank, scal, n, mask, crank);
+          const int oc = bgmv_ochunk(p.out);
+          const int j0 = min(p.out, (int)crank * oc);
+          expand_mma(p, L, sm, w, rank, scal, n, mask, j0, min(p.out, j0 + oc));
         }
         __syncthreads();
       }
@@ -994,9 +1018,11 @@ template <int MODE>
 cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stream,
                         const char** why) {
   BgmvParams p = p_in;
-  bgmv_pick_stages(p.in, p.S, p.R, &p.kb, &p.nst);
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
-  const int npref = (MODE == kModeExpert) ? p.num_experts : p.slots;
+  constexpr bool kSolo = (MODE == kModeExpertSolo);
+  p.kchunk = kSolo ? p.in : bgmv_kchunk(p.in);
+  bgmv_pick_stages(p.kchunk, p.S, p.R, kSolo ? kSoloRingBudget : kRingBudget, &p.kb, &p.nst);
+  const int npref = (MODE == kModeExpert || kSolo) ? p.num_experts : p.slots;
   const BgmvLayout L0 = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst, 0);
   const int ex_bytes = bgmv_ex_stage_bytes(p.out, p.R);
   p.ex_stage = ((MODE == kModeFused || MODE == kModeExpert) &&
@@ -1063,13 +1089,13 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
         *why = "the BGMV kernel does not fit on one SM";
         return cudaErrorInvalidConfiguration;
       }
-      groups = max(1, per_sm * sms / kGroup);
+      groups = kSolo ? per_sm * sms : max(1, per_sm * sms / kGroup);
     }
     std::lock_guard<std::mutex> lk(g_cache_mu);
     if (g_cache_n < 64) g_cache[g_cache_n++] = {dev, MODE, L.total, groups};
   }
   groups = max(1, min(groups, max_items));
-  cfg.gridDim = dim3((unsigned)(groups * kGroup), 1, 1);
+  cfg.gridDim = dim3((unsigned)(kSolo ? groups : groups * kGroup), 1, 1);
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -1084,6 +1110,7 @@ cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream
     case kModeEmbed: return launch_mode<kModeEmbed>(p, max_items, stream, why);
     case kModeGather: return launch_mode<kModeGather>(p, max_items, stream, why);
     case kModeExpert: return launch_mode<kModeExpert>(p, max_items, stream, why);
+    case kModeExpertSolo: return launch_mode<kModeExpertSolo>(p, max_items, stream, why);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -34,8 +34,12 @@ enum BgmvMode : int {
   kModeExpand = 2,  // expand only, h read from global
   kModeEmbed = 3,   // gather + expand (apply_embedding)
   kModeGather = 4,  // gather only (gather_shrink)
-  kModeExpert = 5,  // MoE fold (shrink + expand per (expert chunk, slot))
+  kModeExpert = 5,  // MoE fold (shrink + expand per (expert chunk, slot)), one cluster per chunk
+  kModeExpertSolo = 6,  // MoE fold, one CTA per (expert, slot) pair: shrink over all of in
 };
+
+// Ring budget of the one-CTA-per-pair MoE fold (two CTAs per SM).
+constexpr int kSoloRingBudget = 80 * 1024;
 
 struct BgmvParams {
   const void* x;               // bf16 [rows, in]
@@ -60,6 +64,7 @@ struct BgmvParams {
   int out;
   int num_experts;
   int num_pairs;
+  int kchunk;     // input features one CTA reduces over (multiple of 8)
   int kb;         // input features per stage (multiple of 8)
   int nst;        // stages in the ring (1 or 2)
   int ex_stage;   // 1: the expand operands of an item fit the ring and are staged there
@@ -119,7 +124,8 @@ __host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, in
   L.misc_off = off;
   off += round_up_i(kMiscInts * 4, 128);
   L.ring_off = off;
-  const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpert);
+  const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpert ||
+                     mode == kModeExpertSolo);
   if (ring) off += round_up_i(max(nst * L.stage_bytes, ring_min), 128);
   L.hpart_off = off;
   if (ring) off += 2 * kTT * L.srp * 4;
@@ -132,14 +138,14 @@ __host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, in
   return L;
 }
 
-// Stage width and depth of the staging ring for these shapes (host side).
-inline void bgmv_pick_stages(int in, int S, int R, int* kb, int* nst) {
-  const int kchunk = bgmv_kchunk(in);
+// Stage width and depth of the staging ring for a CTA reducing over kchunk
+// input features (host side).
+inline void bgmv_pick_stages(int kchunk, int S, int R, int budget, int* kb, int* nst) {
   const int rows = S * round_up_i(R, 16) + kTT;
   int k = kchunk < kMaxKB ? kchunk : kMaxKB;
   for (;;) {
     const int n = ceil_div_i(kchunk, k) > 1 ? 2 : 1;
-    if (k <= 64 || n * rows * (2 * k + 16) <= kRingBudget) {
+    if (k <= 64 || n * rows * (2 * k + 16) <= budget) {
       *kb = k;
       *nst = n;
       return;
