@@ -80,15 +80,57 @@ LORA_DEV ShrinkGeom shrink_geom(const BgmvParams& p, int rank, uint32_t crank) {
 // Which staged rows of a stage an issue covers.
 enum RowSet : int { kRowsA = 1, kRowsX = 2, kRowsAll = 3 };
 
-// Warp 0 issues the bulk copies (the TMA engine) of stage kb into ring slot st:
-// the live A rows of adapter w (rows below nrows_a, at i*Rpad + r) and/or the
-// item's x rows (tokens t < n with a valid token, at srp + t), kv input
-// features each.  Their bytes complete on bar; kRowsA only raises the expected
-// bytes, the other sets also arrive (one arrival per phase).  Every address and
-// size is a multiple of 16 bytes (in and the stage offsets are multiples of 8).
+// Every thread issues its share of the 16-byte asynchronous copies of stage kb
+// into ring slot st and commits them as one group: the live A rows of adapter
+// w (rows below nrows_a, at i*Rpad + r) and/or the item's x rows (tokens
+// t < n with a valid token, at srp + t), kv input features each; a warp copies
+// a row.  (Measured on B200: a round of small per-row copies lands sooner
+// through cp.async than through the bulk-copy engine, and the shrink's stages
+// are latency bound.)
 LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
-                         const ShrinkGeom& G, int w, int rank, int n, int kb, int st, int set,
-                         uint64_t* bar) {
+                         const ShrinkGeom& G, int w, int rank, int n, int kb, int st, int set) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int kbase = G.k0 + kb * p.kb;
+  const int cpr = min(p.kb, G.k1 - kbase) >> 3;   // 16-byte chunks per row
+  const int Rpad = round_up_i(p.R, 16);
+  const uint32_t stage = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
+  if ((set & kRowsA) != 0 && G.nrows_a > 0) {
+    // (slice, rank row) of this warp's first A row, advanced 8 rows per step
+    int ai = warp / rank;
+    int ar = warp - ai * rank;
+    for (int row = warp; row < G.nrows_a; row += kBgmvThreads / 32) {
+      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(p.a) +
+                                 ((size_t)w * p.S * p.R + ai * p.R + ar) * p.in + kbase;
+      const uint32_t dst = stage + (uint32_t)((ai * Rpad + ar) * L.row_stride);
+      for (int c = lane; c < cpr; c += 32) cp_async16(dst + c * 16, src + c * 8);
+      ar += kBgmvThreads / 32;
+      while (ar >= rank) {
+        ar -= rank;
+        ++ai;
+      }
+    }
+  }
+  if ((set & kRowsX) != 0) {
+    for (int t = warp; t < n; t += kBgmvThreads / 32) {
+      const int tk = sm.tok[t];
+      if (tk < 0) continue;
+      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)tk * p.in + kbase;
+      const uint32_t dst = stage + (uint32_t)((L.srp + t) * L.row_stride);
+      for (int c = lane; c < cpr; c += 32) cp_async16(dst + c * 16, src + c * 8);
+    }
+  }
+  cp_async_commit();
+}
+
+// Warp 0 issues the same rows as bulk copies (the TMA engine), completing on
+// bar: kRowsA only raises the expected bytes, the other sets also arrive (one
+// arrival per phase).  Used when stage rows are wide (p.bulk_stage): one copy
+// per 1 KB row issues far fewer instructions than 16-byte copies.  Every
+// address and size is a multiple of 16 bytes.
+LORA_DEV void issue_rows_bulk(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                              const ShrinkGeom& G, int w, int rank, int n, int kb, int st,
+                              int set, uint64_t* bar) {
   if (threadIdx.x >= 32) return;
   const int lane = threadIdx.x;
   const int kbase = G.k0 + kb * p.kb;
@@ -96,9 +138,7 @@ LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   const int Rpad = round_up_i(p.R, 16);
   uint8_t* stage = sm.ring + st * L.stage_bytes;
   const bool want_a = (set & kRowsA) != 0 && G.nrows_a > 0;
-  const bool want_x = (set & kRowsX) != 0;
-  const int t = lane;
-  const bool xrow = want_x && t < n && sm.tok[t] >= 0;
+  const bool xrow = (set & kRowsX) != 0 && lane < n && sm.tok[lane] >= 0;
   const uint32_t xmask = __ballot_sync(0xffffffffu, xrow);
   if (lane == 0) {
     fence_proxy_async_smem();
@@ -111,7 +151,6 @@ LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   }
   __syncwarp();
   if (want_a) {
-    // (slice, rank row) of this lane's first A row, advanced 32 rows per step
     int ai = lane / rank;
     int ar = lane - ai * rank;
     for (int row = lane; row < G.nrows_a; row += 32) {
@@ -127,33 +166,47 @@ LORA_DEV void issue_rows(const BgmvParams& p, const BgmvLayout& L, const Smem& s
   }
   if (xrow) {
     const __nv_bfloat16* src =
-        reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)sm.tok[t] * p.in + kbase;
-    bulk_g2s(stage + (L.srp + t) * L.row_stride, src, rbytes, bar);
+        reinterpret_cast<const __nv_bfloat16*>(p.x) + (size_t)sm.tok[lane] * p.in + kbase;
+    bulk_g2s(stage + (L.srp + lane) * L.row_stride, src, rbytes, bar);
   }
 }
 
 // Warp-uniform bounded wait for phase `parity` of bar; on timeout raises
 // LORA_FLAG_TIMEOUT and waits once more (bounded) so that no copy is still in
-// flight when the shared memory is reused.  Returns false on timeout.
-LORA_DEV bool wait_stage(uint64_t* bar, uint32_t parity, uint32_t* flags) {
-  bool ok = true;
+// flight when the shared memory is reused.
+LORA_DEV void wait_stage(uint64_t* bar, uint32_t parity, uint32_t* flags) {
   if ((threadIdx.x & 31) == 0) {
-    ok = mbar_wait(bar, parity);
-    if (!ok) {
+    if (!mbar_wait(bar, parity)) {
       raise_flag(flags, LORA_FLAG_TIMEOUT);
       mbar_wait(bar, parity);
     }
   }
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+}
+
+// Copies of the shrink's stages: per-thread cp.async groups, or bulk copies
+// on the ring slots' mbarriers (sbar, phase parity bit st of sph).
+struct StageCopies {
+  bool bulk;
+  uint64_t* sbar;
+  uint32_t sph;
+};
+
+LORA_DEV void issue_stage(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
+                          const ShrinkGeom& G, int w, int rank, int n, int kb, int st, int set,
+                          StageCopies& sc) {
+  if (sc.bulk)
+    issue_rows_bulk(p, L, sm, G, w, rank, n, kb, st, set, &sc.sbar[st]);
+  else
+    issue_rows(p, L, sm, G, w, rank, n, kb, st, set);
 }
 
 // MMAs of the shrink over this CTA's input features into hpart[t * srp +
 // i*Rpad + r] (every 16-row tile holding a live row, t < 8*ceil(n/8)).  The
-// caller has issued the A rows of stage 0 (kRowsA on sbar[0]); this issues the
-// rest.  sph holds the phase parity of each ring slot's barrier (bit st).
+// caller has issued the A rows of stage 0 (kRowsA); this issues the rest.
 LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
                              const ShrinkGeom& G, int w, int rank, int n, float* hpart,
-                             uint64_t* sbar, uint32_t& sph) {
+                             StageCopies& sc) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -171,13 +224,18 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
     for (int q = 0; q < 4; ++q) acc[c][q] = 0.f;
 
   if (G.nkb > 0) {
-    issue_rows(p, L, sm, G, w, rank, n, 0, 0, kRowsX, &sbar[0]);
-    if (G.nkb > 1 && p.nst == 2) issue_rows(p, L, sm, G, w, rank, n, 1, 1, kRowsAll, &sbar[1]);
+    issue_stage(p, L, sm, G, w, rank, n, 0, 0, kRowsX, sc);
+    if (G.nkb > 1 && p.nst == 2) issue_stage(p, L, sm, G, w, rank, n, 1, 1, kRowsAll, sc);
   }
   for (int kb = 0; kb < G.nkb; ++kb) {
     const int st = kb % p.nst;
-    wait_stage(&sbar[st], (sph >> st) & 1u, p.flags);
-    sph ^= 1u << st;
+    if (sc.bulk) {
+      wait_stage(&sc.sbar[st], (sc.sph >> st) & 1u, p.flags);
+      sc.sph ^= 1u << st;
+    } else {
+      if (kb + 1 < G.nkb && p.nst == 2) cp_async_wait<1>(); else cp_async_wait<0>();
+      __syncthreads();
+    }
     const int kv = min(p.kb, G.k1 - (G.k0 + kb * p.kb));
     const int nks = ceil_div_i(kv, 16);
     const uint32_t stage_addr = smem_u32(sm.ring) + (uint32_t)(st * L.stage_bytes);
@@ -207,8 +265,7 @@ LORA_DEV void shrink_partial(const BgmvParams& p, const BgmvLayout& L, const Sme
       }
     }
     __syncthreads();
-    if (kb + p.nst < G.nkb)
-      issue_rows(p, L, sm, G, w, rank, n, kb + p.nst, st, kRowsAll, &sbar[st]);
+    if (kb + p.nst < G.nkb) issue_stage(p, L, sm, G, w, rank, n, kb + p.nst, st, kRowsAll, sc);
   }
 
   const int g8 = lane >> 2;
@@ -723,15 +780,17 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   // the cluster reduces h; ebar counts their bytes (one phase per use).
   const bool staged = kExpands && kClustered && p.ex_stage != 0;
   uint64_t* ebar = reinterpret_cast<uint64_t*>(smem_raw);
-  // Ring slots' barriers: the bulk copies of a shrink stage complete on them.
-  uint64_t* sbar = ebar + 1;
-  uint32_t sph = 0;
   const ExStage X = ex_stage_carve(sm, p);
   uint32_t ephase = 0;
-  if (tid == 0 && (staged || kClustered || kSolo)) {
+  // Shrink stage copies: bulk copies complete on the ring slots' barriers.
+  StageCopies sc;
+  sc.bulk = p.bulk_stage != 0;
+  sc.sbar = ebar + 1;
+  sc.sph = 0;
+  if (tid == 0 && (staged || sc.bulk)) {
     mbar_init(ebar, 1);
-    mbar_init(&sbar[0], 1);
-    mbar_init(&sbar[1], 1);
+    mbar_init(&sc.sbar[0], 1);
+    mbar_init(&sc.sbar[1], 1);
     fence_mbar_init();
   }
 
@@ -835,7 +894,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       if (kClustered) {
         // the A rows do not depend on the tokens: start them while the reads land
         G = shrink_geom(p, rank, crank);
-        if (G.nkb > 0) issue_rows(p, L, sm, G, s, rank, 0, 0, 0, kRowsA, &sbar[0]);
+        if (G.nkb > 0) issue_stage(p, L, sm, G, s, rank, 0, 0, 0, kRowsA, sc);
       }
       if (tid < kTT) {
         int id = -1;
@@ -865,7 +924,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, s, n, rowmask, crank);
       if (kClustered) {
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
-        shrink_partial(p, L, sm, G, s, rank, n, hp, sbar, sph);
+        shrink_partial(p, L, sm, G, s, rank, n, hp, sc);
         if (staged) stage_expand(p, sm, X, s, n, rowmask, crank, ebar);
         cluster_sync();
         produce_h<kFromCluster>(p, L, sm, hp, s, rank, n, rowmask, kExpands,
@@ -964,13 +1023,13 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         const int rank = mine ? p.ranks[sl] : 0;
         const float scal = mine ? p.scalings[sl] : 0.f;
         const ShrinkGeom G = shrink_geom(p, rank, kSolo ? 0u : crank);
-        if (G.nkb > 0 && rank > 0) issue_rows(p, L, sm, G, w, rank, 0, 0, 0, kRowsA, &sbar[0]);
+        if (G.nkb > 0 && rank > 0) issue_stage(p, L, sm, G, w, rank, 0, 0, 0, kRowsA, sc);
         if (tid < kTT) sm.tok[tid] = (tid < n) ? sm.sub_rows[q * kTT + tid] : -1;
         __syncthreads();
         const uint32_t mask = (n >= 32) ? 0xffffffffu : ((1u << n) - 1u);
         if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, w, n, mask, crank);
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
-        shrink_partial(p, L, sm, G, w, rank, n, hp, sbar, sph);
+        shrink_partial(p, L, sm, G, w, rank, n, hp, sc);
         if (kSolo) {
           __syncthreads();
           produce_h<kFromLocal>(p, L, sm, hp, w, rank, n, mask, true, false, 0);
@@ -1030,6 +1089,9 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
                    ? 1
                    : 0;
   const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst, p.ex_stage ? ex_bytes : 0);
+  // Wide stage rows (1 KB) go as one bulk copy each; narrower ones as 16-byte
+  // cp.async copies, which land sooner for small rounds.
+  p.bulk_stage = (p.kb >= 512 && (kClustered || kSolo)) ? 1 : 0;
   auto kern = bgmv_kernel<MODE>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
