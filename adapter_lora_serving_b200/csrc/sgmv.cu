@@ -11,9 +11,10 @@
 //         memory, updated with bf16_rne(y + scaling * D) and stored with
 //         coalesced row writes.
 // Both kernels are persistent (one CTA per SM over a contiguous run of work
-// units) and warp-specialised: warp 0 loads, warp 1 issues MMAs (one thread),
-// the other warps drain TMEM (shrink: 4; expand: 16, each 32 rows x 32
-// columns).  Every wait is bounded; on timeout the CTA raises
+// units) and warp-specialised: warp 1 issues MMAs (one thread); the shrink
+// copies x with 4 warps (0 and 6-8, warp 0 also starts the A tiles) and
+// drains TMEM with 4; the expand loads B with warp 0 and drains TMEM with 16
+// (each 32 rows x 32 columns).  Every wait is bounded; on timeout the CTA raises
 // LORA_FLAG_TIMEOUT, stops, frees its TMEM and exits.
 //
 // Sources: mstar.engine.resources.lora.backend (LoraBackend.shrink,
@@ -31,7 +32,8 @@ namespace lora {
 
 namespace {
 
-constexpr int kSgThreads = 192;   // shrink: 6 warps
+constexpr int kSgXWarps = 4;      // shrink: warps that copy x rows (warp 0 and warps 6..8)
+constexpr int kSgThreads = 32 * (6 + kSgXWarps - 1);   // shrink: 9 warps
 constexpr int kExEpiWarps = 16;   // expand epilogue: 4 TMEM lane quarters x 4 column groups
 constexpr int kExThreads = 32 * (2 + kExEpiWarps);   // expand: producer, MMA, epilogue
 constexpr int kNY = 3;            // y staging buffers (prefetch two units ahead)
@@ -472,7 +474,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
 
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) {
-      mbar_init(&full[i], 33);   // 32 cp.async arrivals + 1 expect_tx arrival
+      mbar_init(&full[i], 32 * kSgXWarps + 1);   // cp.async arrivals + 1 expect_tx arrival
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -511,8 +513,16 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
     kb1 = min(nkb_total, kb0 + p.kb_per_split);
   };
 
-  if (warp == 0) {
-    // ---------------- producer: x rows by cp.async, A rows by tensor TMA ----------------
+  if (warp == 0 || warp >= 6) {
+    // ---------------- producers: x rows by cp.async (4 warps), A rows by tensor TMA (warp 0) ----
+    // Producer thread pt (0..127) copies 16-byte chunk c = pt % 8 of the tile
+    // rows pt / 8 + 16 j (j < 8): eight lanes cover a 128-byte row segment,
+    // and the chunk's swizzled position depends on the row only through
+    // row % 8 = (pt / 8) % 8, fixed for the thread.
+    const int pt = (warp == 0 ? 0 : warp - 5) * 32 + lane;
+    const int c = pt & 7;
+    const int r0 = pt >> 3;
+    const uint32_t cswz = (uint32_t)(((c ^ (r0 & 7)) << 4));
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(p.x);
     int g = 0;  // stages issued
     for (int k = 0; k < nloc; ++k) {
@@ -520,19 +530,19 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
       unit_geom(u0 + k, s, p0, n, kb0, kb1, ks);
       const int rank = p.ranks[s];
       const int K0 = ceil_div_i(rank, 16) * 16;
-      int trow[4];
+      int trow[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int mm = lane + 32 * q;
+      for (int j2 = 0; j2 < 8; ++j2) {
+        const int mm = r0 + 16 * j2;
         int t = -1;
         if (mm < n) {
           t = p.token_order[p0 + mm];
           if (t < 0 || t >= p.T) {
-            if (ks == 0) raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
+            if (ks == 0 && c == 0) raise_flag(p.flags, LORA_FLAG_BAD_TOKEN);
             t = -1;
           }
         }
-        trow[q] = t;
+        trow[j2] = t;
       }
       bool ok = true;
       for (int kb = kb0; kb < kb1; ++kb, ++g) {
@@ -543,7 +553,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
         }
         uint8_t* xt = ring + st * kStage;
         uint8_t* at = xt + kXTile;
-        if (lane == 0) {
+        if (warp == 0 && lane == 0) {
           const int groups = ceil_div_i(rank, 16);
           mbar_arrive_expect_tx(&full[st], (uint32_t)(p.S * groups * 16 * 128));
           for (int i = 0; i < p.S; ++i)
@@ -551,17 +561,15 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
               tma_load_2d(at + (i * K0 + 16 * q) * 128, &tmap_a, kb * kKBLK,
                           s * SR + i * p.R + 16 * q, &full[st]);
         }
-        const int kbase = kb * kKBLK;
+        const int kcol = kb * kKBLK + c * 8;
+        const bool cok = kcol < p.in;
+        const uint32_t xbase = smem_u32(xt) + cswz;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int mm = lane + 32 * q;
-          const int t = trow[q];
-          const __nv_bfloat16* src = xb + (size_t)(t >= 0 ? t : 0) * p.in + kbase;
-          for (int c = 0; c < 8; ++c) {
-            const bool valid = t >= 0 && kbase + c * 8 < p.in;
-            cp_async16_zfill(smem_u32(xt) + kmajor_offset(mm, c * 8, 128), valid ? src + c * 8 : xb,
-                             valid);
-          }
+        for (int j2 = 0; j2 < 8; ++j2) {
+          const int t = trow[j2];
+          const bool valid = t >= 0 && cok;
+          cp_async16_zfill(xbase + (uint32_t)((r0 + 16 * j2) * 128),
+                           valid ? xb + (size_t)t * p.in + kcol : xb, valid);
         }
         cp_async_arrive_noinc(&full[st]);
       }
