@@ -126,6 +126,8 @@ const char* lora_status_string(lora_status status) {
 
 const char* lora_last_error(void) { return g_last_error; }
 
+int32_t lora_set_launch_overlap(int32_t enable) { return lora::bgmv_set_overlap(enable); }
+
 const char* lora_version(void) { return "lora_delta 0.1.0 sm_100a"; }
 
 int32_t lora_resolve_regime(int32_t op, int32_t T, int32_t slots, int32_t R, int32_t num_slices) {

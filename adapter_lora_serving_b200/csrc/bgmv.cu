@@ -16,6 +16,7 @@
 // expand_fused, apply_linear_, gather_shrink, apply_) and
 // spark_model/lora/expert_apply.rs (apply_expert_lora_sorted, with the
 // per-(slot, expert) grouping the page plans as its grouped BGMV kernel).
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -771,6 +772,11 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
   constexpr bool kScaled = (MODE == kModeFused || MODE == kModeExpand || MODE == kModeEmbed || kMoE);
   constexpr bool kExpands = kScaled;
   extern __shared__ __align__(128) uint8_t smem_raw[];
+  // With a programmatic launch edge (fused mode only) the next kernel may
+  // start its CTAs as ours finish, and ours read x and y only after the
+  // preceding kernel completed (grid_dep_wait below); without one both are
+  // no-ops.
+  if (MODE == kModeFused) grid_dep_launch_dependents();
   const int npref = kMoE ? p.num_experts : p.slots;
   const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst,
                                    p.ex_stage ? bgmv_ex_stage_bytes(p.out, p.R) : 0);
@@ -896,6 +902,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         G = shrink_geom(p, rank, crank);
         if (G.nkb > 0) issue_stage(p, L, sm, G, s, rank, 0, 0, 0, kRowsA, sc);
       }
+      if (MODE == kModeFused && iter == 0) grid_dep_wait();   // x and y from here on
       if (tid < kTT) {
         int id = -1;
         if (tid < n && p0 + tid >= 0 && p0 + tid < p.T) {
@@ -1063,6 +1070,8 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
 
 namespace {
 
+std::atomic<int> g_overlap{0};
+
 // Per (device, mode, shared-memory size): the number of work groups one launch
 // uses.  Filled on the first call with those shapes; later calls (and calls
 // during stream capture) only read it.
@@ -1098,7 +1107,7 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
   if (err != cudaSuccess) return err;
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(kBgmvThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = stream;
@@ -1109,6 +1118,12 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+  }
+  if (MODE == kModeFused && g_overlap.load(std::memory_order_relaxed) != 0) {
+    attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs += 1;
   }
 
   int groups = -1;
@@ -1162,6 +1177,8 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
 }
 
 }  // namespace
+
+int bgmv_set_overlap(int enable) { return g_overlap.exchange(enable != 0 ? 1 : 0); }
 
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,
                         const char** why) {

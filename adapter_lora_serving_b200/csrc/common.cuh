@@ -142,6 +142,17 @@ LORA_DEV void cp_async_wait() {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch (no-ops when the launch has no such edge)
+// ---------------------------------------------------------------------------
+
+// Lets the next kernel in the stream start launching its CTAs.
+LORA_DEV void grid_dep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the preceding kernel has completed and its writes are visible.
+LORA_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters
 // ---------------------------------------------------------------------------
 

@@ -155,6 +155,10 @@ inline void bgmv_pick_stages(int kchunk, int S, int R, int budget, int* kb, int*
   }
 }
 
+// Process-wide opt-in to programmatic dependent launch of the fused BGMV
+// kernel (lora_set_launch_overlap).
+int bgmv_set_overlap(int enable);
+
 // Launchers (bgmv.cu).  Return a cudaError_t from the launch.
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,
                         const char** why);

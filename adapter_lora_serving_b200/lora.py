@@ -62,6 +62,7 @@ _SIGS = [
     ("lora_plan_tile", _I, [_I, _I]),
     ("lora_plan_linear", _I, [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
     ("lora_plan_expert", _I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
+    ("lora_set_launch_overlap", _I, [_I]),
     ("lora_status_string", ctypes.c_char_p, [_I]),
     ("lora_last_error", ctypes.c_char_p, []),
     ("lora_version", ctypes.c_char_p, []),
@@ -213,6 +214,12 @@ def lora_plan_expert(expert_offsets, pair_index, rows_cap, num_experts, slots, m
     _check(load().lora_plan_expert(_ptr(expert_offsets), _ptr(pair_index), rows_cap,
                                    num_experts, slots, max_rows, _ptr(plan_out), plan_cap,
                                    _ptr(plan_count), _ptr(err_flags), _stream(stream)))
+
+
+def lora_set_launch_overlap(enable):
+    """Opt in or out of overlapping the fused few-tokens kernel's start with
+    the preceding kernel in the stream; returns the previous setting."""
+    return int(load().lora_set_launch_overlap(1 if enable else 0))
 
 
 def lora_version():

@@ -253,6 +253,21 @@ LORA_API lora_status lora_plan_expert(const int32_t* expert_offsets, const int32
                              int32_t max_rows, int32_t* plan_out, int32_t plan_cap,
                              int32_t* plan_count, uint32_t* err_flags, void* stream);
 
+/*
+ * lora_set_launch_overlap -- opt in (enable != 0) or out of overlapping the
+ * start of lora_apply_linear's few-tokens (BGMV) kernel with the end of the
+ * kernel that precedes it in the stream (CUDA programmatic dependent launch;
+ * captured into CUDA graphs as a programmatic edge).  With it on, that kernel
+ * plans its work items and starts loading the adapters' A rows before the
+ * preceding kernel has finished, and reads x and y only after it has finished
+ * and its writes are visible.  Contract while enabled: the kernel preceding a
+ * lora_apply_linear call in its stream does not write a, b, ranks, scalings,
+ * token_order or slot_indptr of that call.  Process-wide; off by default;
+ * takes effect for launches issued after the call.  Returns the previous
+ * setting.
+ */
+LORA_API int32_t lora_set_launch_overlap(int32_t enable);
+
 LORA_API const char* lora_status_string(lora_status status);
 LORA_API const char* lora_last_error(void);
 /* Library version, e.g. "lora_delta 0.1.0 sm_100a". */

@@ -405,3 +405,65 @@ def test_workload_moe_full():
     gu, dn = W.moe_expert(0)
     for m in (gu, dn):
         _check_moe(m, what=m.name)
+
+
+# ---------------------------------------------------------------------------
+# Launch overlap (programmatic dependent launch) between dependent calls
+# ---------------------------------------------------------------------------
+
+def _chain_problems():
+    # Three few-tokens fused calls on one y: each reads the y the previous
+    # call wrote, with its own x, adapters and slot layout.
+    ps = [W.random_linear(900 + k, 256, 512, (256, 128, 64), 12, 16, ranks=None,
+                          dead_frac=0.1) for k in range(3)]
+    return ps
+
+
+def _oracle_chain(ps, y0):
+    y = y0
+    for p in ps:
+        y_ref, _, _ = _oracle_linear(p, y)
+        y = W.f32_to_bf16_bits(y_ref)
+    return y
+
+
+@pytest.mark.parametrize("graph", [False, True], ids=["stream", "graph"])
+def test_launch_overlap_dependent_chain(graph):
+    """With the overlap on, each call still sees the y its predecessor wrote
+    (x and y are read only after the preceding kernel completed)."""
+    t = torch()
+    ps = _chain_problems()
+    devs = [LinearDev(p) for p in ps]
+    y = devs[0].y
+    y0 = host_bits(y).copy()
+    prev = L.lora_set_launch_overlap(1)
+    try:
+        def run():
+            for d in devs:
+                p = d.p
+                L.lora_apply_linear(d.x, y, d.a, d.b, d.ranks, d.scalings, d.token_order,
+                                    d.slot_indptr, p.T, p.n_in, p.slots, p.R, p.out_slices,
+                                    regime=L.LORA_REGIME_BGMV, err_flags=d.flags)
+        if graph:
+            run()                                   # warm the launch caches outside capture
+            t.cuda.synchronize()
+            y.copy_(t.from_numpy(y0.view(np.int16).copy()).view(t.bfloat16).cuda())
+            g = t.cuda.CUDAGraph()
+            with t.cuda.graph(g):
+                run()
+            y.copy_(t.from_numpy(y0.view(np.int16).copy()).view(t.bfloat16).cuda())
+            g.replay()
+        else:
+            run()
+        t.cuda.synchronize()
+    finally:
+        L.lora_set_launch_overlap(prev)
+    ref = _oracle_chain(ps, y0)
+    assert_close(_f64(host_bits(y)), _f64(ref), "chain")
+    assert all(read_flags(d.flags) == 0 for d in devs)
+
+
+def test_launch_overlap_setting_roundtrip():
+    prev = L.lora_set_launch_overlap(1)
+    assert L.lora_set_launch_overlap(0) == 1
+    assert L.lora_set_launch_overlap(prev) == 0
