@@ -1179,6 +1179,7 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
 }  // namespace
 
 int bgmv_set_overlap(int enable) { return g_overlap.exchange(enable != 0 ? 1 : 0); }
+bool launch_overlap_enabled() { return g_overlap.load(std::memory_order_relaxed) != 0; }
 
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,
                         const char** why) {

@@ -156,8 +156,9 @@ inline void bgmv_pick_stages(int kchunk, int S, int R, int budget, int* kb, int*
 }
 
 // Process-wide opt-in to programmatic dependent launch of the fused BGMV
-// kernel (lora_set_launch_overlap).
+// kernel and the SGMV kernels (lora_set_launch_overlap).
 int bgmv_set_overlap(int enable);
+bool launch_overlap_enabled();
 
 // Launchers (bgmv.cu).  Return a cudaError_t from the launch.
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,

@@ -146,6 +146,10 @@ struct UnitCursor {
 __global__ void __launch_bounds__(kExThreads, 1)
 sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParams p) {
   extern __shared__ uint8_t sg_smem_raw[];
+  // Programmatic launch edge (when the caller opted in): let the next kernel
+  // start as CTAs finish; only the epilogue, which reads y, h and ids and
+  // writes y, waits for the preceding kernel.  No-ops otherwise.
+  grid_dep_launch_dependents();
   const uint32_t raw = smem_u32(sg_smem_raw);
   uint8_t* base = sg_smem_raw + (align1024(raw) - raw);
   uint64_t* bfull = reinterpret_cast<uint64_t*>(base);
@@ -262,6 +266,7 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
     }
   } else {
     // ---------------- epilogue: warps 2..17 ----------------
+    grid_dep_wait();
     // Warp w reads TMEM lanes 32*(w%4).. (one token row per thread) and owns
     // the 32 columns [32 cg, 32 cg + 32) of the unit, cg = (w - 2) / 4.
     const int quarter = warp & 3;
@@ -451,6 +456,9 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
 __global__ void __launch_bounds__(kSgThreads, 1)
 sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParams p) {
   extern __shared__ uint8_t sg_smem_raw[];
+  // Programmatic launch edge (when the caller opted in): the producers (x)
+  // and the epilogue (writes h) wait for the preceding kernel.
+  grid_dep_launch_dependents();
   const uint32_t raw = smem_u32(sg_smem_raw);
   uint8_t* base = sg_smem_raw + (align1024(raw) - raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(base);
@@ -515,6 +523,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
 
   if (warp == 0 || warp >= 6) {
     // ---------------- producers: x rows by cp.async (4 warps), A rows by tensor TMA (warp 0) ----
+    grid_dep_wait();
     // Producer thread pt (0..127) copies 16-byte chunk c = pt % 8 of the tile
     // rows pt / 8 + 16 j (j < 8): eight lanes cover a 128-byte row segment,
     // and the chunk's swizzled position depends on the row only through
@@ -619,6 +628,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
     }
   } else {
     // ---------------- epilogue ----------------
+    grid_dep_wait();
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
@@ -730,6 +740,27 @@ cudaError_t dev_info(DevInfo** out) {
   return cudaSuccess;
 }
 
+// Launch with a programmatic stream-serialization edge when the process opted
+// in (lora_set_launch_overlap), else as a plain launch.
+template <typename P>
+cudaError_t launch_overlapped(void (*kern)(const CUtensorMap, const P), int grid, int threads,
+                              size_t smem, cudaStream_t stream, const CUtensorMap& map,
+                              const P& p) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  if (launch_overlap_enabled()) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, map, p);
+}
+
 size_t expand_smem(int slots, int span) {
   const size_t pre = ((size_t)(slots + 1) * 4 + 1023) / 1024 * 1024;
   return 1024 + 1024 + pre + 2 * (size_t)kTM * span + (size_t)kNB * kBN * span +
@@ -792,8 +823,7 @@ cudaError_t sgmv_shrink_launch(const void* x, const void* a, float* h, const int
   }
   const int units = (slots + ceil_div_i(T, kTM)) * p.ksplit;
   const int grid = max(1, min(d->sms, units));
-  sgmv_shrink_kernel<<<grid, kSgThreads, smem, stream>>>(map, p);
-  return cudaGetLastError();
+  return launch_overlapped(sgmv_shrink_kernel, grid, kSgThreads, smem, stream, map, p);
 }
 
 int sgmv_shrink_splits(int T, int slots, int in) {
@@ -838,8 +868,7 @@ cudaError_t sgmv_expand_launch(void* y, const float* h, int ksplit, const int* i
   }
   const long long units = (long long)(slots + ceil_div_i(T, kTM)) * nchunk;
   const int grid = (int)max(1LL, min((long long)d->sms, units));
-  sgmv_expand_kernel<<<grid, kExThreads, smem, stream>>>(map, p);
-  return cudaGetLastError();
+  return launch_overlapped(sgmv_expand_kernel, grid, kExThreads, smem, stream, map, p);
 }
 
 }  // namespace lora

@@ -255,16 +255,17 @@ LORA_API lora_status lora_plan_expert(const int32_t* expert_offsets, const int32
 
 /*
  * lora_set_launch_overlap -- opt in (enable != 0) or out of overlapping the
- * start of lora_apply_linear's few-tokens (BGMV) kernel with the end of the
- * kernel that precedes it in the stream (CUDA programmatic dependent launch;
- * captured into CUDA graphs as a programmatic edge).  With it on, that kernel
- * plans its work items and starts loading the adapters' A rows before the
- * preceding kernel has finished, and reads x and y only after it has finished
- * and its writes are visible.  Contract while enabled: the kernel preceding a
- * lora_apply_linear call in its stream does not write a, b, ranks, scalings,
- * token_order or slot_indptr of that call.  Process-wide; off by default;
- * takes effect for launches issued after the call.  Returns the previous
- * setting.
+ * start of a kernel with the end of the kernel that precedes it in the stream
+ * (CUDA programmatic dependent launch; captured into CUDA graphs as a
+ * programmatic edge), for lora_apply_linear (both regimes) and
+ * lora_apply_embedding / lora_shrink / lora_expand in the SGMV regime.  With it
+ * on, a kernel plans its work items and starts loading adapter rows before the
+ * preceding kernel has finished; it reads x, y, h and ids, and writes any
+ * output or workspace, only after that kernel has finished and its writes are
+ * visible.  Contract while enabled: the kernel preceding such a call in its
+ * stream does not write a, b, ranks, scalings, token_order or slot_indptr of
+ * that call.  Process-wide; off by default; takes effect for launches issued
+ * after the call.  Returns the previous setting.
  */
 LORA_API int32_t lora_set_launch_overlap(int32_t enable);
 

@@ -411,12 +411,14 @@ def test_workload_moe_full():
 # Launch overlap (programmatic dependent launch) between dependent calls
 # ---------------------------------------------------------------------------
 
-def _chain_problems():
-    # Three few-tokens fused calls on one y: each reads the y the previous
-    # call wrote, with its own x, adapters and slot layout.
-    ps = [W.random_linear(900 + k, 256, 512, (256, 128, 64), 12, 16, ranks=None,
-                          dead_frac=0.1) for k in range(3)]
-    return ps
+def _chain_problems(regime):
+    # Three fused calls on one y: each reads the y the previous call wrote,
+    # with its own x, adapters and slot layout.
+    if regime == L.LORA_REGIME_SGMV:
+        return [W.random_linear(910 + k, 1200, 256, (128, 64), 4, 32, ranks=[32, 16, 8, 32],
+                                dead_frac=0.05) for k in range(3)]
+    return [W.random_linear(900 + k, 256, 512, (256, 128, 64), 12, 16, ranks=None,
+                            dead_frac=0.1) for k in range(3)]
 
 
 def _oracle_chain(ps, y0):
@@ -427,13 +429,18 @@ def _oracle_chain(ps, y0):
     return y
 
 
+@pytest.mark.parametrize("regime", REGIMES)
 @pytest.mark.parametrize("graph", [False, True], ids=["stream", "graph"])
-def test_launch_overlap_dependent_chain(graph):
+def test_launch_overlap_dependent_chain(regime, graph):
     """With the overlap on, each call still sees the y its predecessor wrote
-    (x and y are read only after the preceding kernel completed)."""
+    (x, y and h are read only after the preceding kernel completed), and calls
+    sharing one workspace do not overwrite h while it is being read."""
     t = torch()
-    ps = _chain_problems()
+    ps = _chain_problems(regime)
     devs = [LinearDev(p) for p in ps]
+    ws_bytes = max(L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R,
+                                          p.num_slices, regime) for p in ps)
+    ws = t.zeros(max(ws_bytes, 16) // 4, dtype=t.float32, device="cuda")
     y = devs[0].y
     y0 = host_bits(y).copy()
     prev = L.lora_set_launch_overlap(1)
@@ -443,7 +450,8 @@ def test_launch_overlap_dependent_chain(graph):
                 p = d.p
                 L.lora_apply_linear(d.x, y, d.a, d.b, d.ranks, d.scalings, d.token_order,
                                     d.slot_indptr, p.T, p.n_in, p.slots, p.R, p.out_slices,
-                                    regime=L.LORA_REGIME_BGMV, err_flags=d.flags)
+                                    regime=regime, workspace=ws if ws_bytes else None,
+                                    workspace_bytes=ws_bytes, err_flags=d.flags)
         if graph:
             run()                                   # warm the launch caches outside capture
             t.cuda.synchronize()
