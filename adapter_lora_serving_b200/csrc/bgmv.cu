@@ -1,16 +1,18 @@
 // BGMV regime of the LoRA delta path (few tokens per slot): one thread-block
-// cluster per work item of at most kTT tokens of one slot (or of one MoE
-// expert chunk and slot).
+// cluster of kGroup CTAs per work item of at most kTT tokens of one slot; the
+// MoE fold runs one CTA per kTT-row chunk of an expert instead.
 //
 // Shrink: each CTA of the cluster owns 1/kGroup of the input features.  The
-// slot's live A rows and the item's x rows are staged in shared memory by
-// coalesced 16-byte asynchronous copies and feed m16n8k16 warp MMAs
-// (fp32 accumulate).  The kGroup partial h tiles are summed in a fixed order
-// through distributed shared memory, so every CTA holds the same full h and
-// h never leaves the chip.
-// Expand: each CTA owns 1/kGroup of the output columns; a thread owns a column
-// pair and does the rank-r dot products for every token of the item in fp32,
-// then y = bf16_rne(y + scaling * acc) with coalesced 4-byte stores.
+// slot's live A rows and the item's x rows are staged in padded shared-memory
+// rows (16-byte cp.async, or one bulk copy per 1 KB row) and feed m16n8k16
+// warp MMAs (fp32 accumulate).  The kGroup partial h tiles are summed in a
+// fixed order through distributed shared memory, so every CTA holds the same
+// full h and h never leaves the chip.
+// Expand: each CTA owns 1/kGroup of the output columns.  For the fused path
+// the slot's B columns and the item's y rows are bulk-copied into the idle
+// staging ring while the cluster reduces h; m16n8k16 MMAs (columns as M,
+// tokens as N, h = hi + lo in bf16) update y in shared memory, which is then
+// written back with coalesced 16-byte stores.  y = bf16_rne(y + scaling * acc).
 //
 // Sources: mstar.engine.resources.lora.backend (LoraBackend.shrink,
 // expand_fused, apply_linear_, gather_shrink, apply_) and
@@ -766,9 +768,9 @@ LORA_DEV void expand_after_stage(const BgmvParams& p, const BgmvLayout& L, const
 
 template <int MODE>
 __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams p) {
-  constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
+  constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink);
   constexpr bool kSolo = (MODE == kModeExpertSolo);
-  constexpr bool kMoE = (MODE == kModeExpert || kSolo);
+  constexpr bool kMoE = kSolo;
   constexpr bool kScaled = (MODE == kModeFused || MODE == kModeExpand || MODE == kModeEmbed || kMoE);
   constexpr bool kExpands = kScaled;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -956,7 +958,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       }
       __syncthreads();
     } else {
-      // ---- MoE item: chunk of one expert's rows, split by slot ----
+      // ---- MoE item (one CTA): chunk of one expert's rows, split by slot ----
       const int E = p.num_experts;
       const int e = find_segment(sm.prefix, E, item);
       const int chunk = item - sm.prefix[e];
@@ -1016,47 +1018,25 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         }
       }
       __syncthreads();
-      const int my_nsub = *nsub_slot;
-      int nsub = my_nsub;
-      if (!kSolo) {
-        cluster_sync();
-        nsub = dsmem_ld_s32(dsmem_addr(nsub_slot, 0));
-      }
+      const int nsub = *nsub_slot;
       for (int q = 0; q < nsub; ++q) {
-        const bool mine = q < my_nsub;
-        const int sl = mine ? sm.sub_s[q] : 0;
-        const int w = mine ? sm.sub_p[q] : 0;
-        const int n = mine ? sm.sub_cnt[q] : 0;
-        const int rank = mine ? p.ranks[sl] : 0;
-        const float scal = mine ? p.scalings[sl] : 0.f;
-        const ShrinkGeom G = shrink_geom(p, rank, kSolo ? 0u : crank);
+        const int sl = sm.sub_s[q];
+        const int w = sm.sub_p[q];
+        const int n = sm.sub_cnt[q];
+        const int rank = p.ranks[sl];
+        const float scal = p.scalings[sl];
+        const ShrinkGeom G = shrink_geom(p, rank, 0u);
         if (G.nkb > 0 && rank > 0) issue_stage(p, L, sm, G, w, rank, 0, 0, 0, kRowsA, sc);
         if (tid < kTT) sm.tok[tid] = (tid < n) ? sm.sub_rows[q * kTT + tid] : -1;
         __syncthreads();
         const uint32_t mask = (n >= 32) ? 0xffffffffu : ((1u << n) - 1u);
-        if (staged && (tid >> 5) == 1) prefetch_expand(p, sm, w, n, mask, crank);
         float* hp = sm.hpart + (size_t)hpar * kTT * L.srp;
         shrink_partial(p, L, sm, G, w, rank, n, hp, sc);
-        if (kSolo) {
-          __syncthreads();
-          produce_h<kFromLocal>(p, L, sm, hp, w, rank, n, mask, true, false, 0);
-        } else {
-          if (staged) stage_expand(p, sm, X, w, n, mask, crank, ebar);
-          cluster_sync();
-          produce_h<kFromCluster>(p, L, sm, hp, w, rank, n, mask, true, false, crank);
-        }
+        __syncthreads();
+        produce_h<kFromLocal>(p, L, sm, hp, w, rank, n, mask, true, false, 0);
         hpar ^= 1;
         __syncthreads();
-        if (staged) {
-          expand_after_stage(p, L, sm, X, ebar, ephase, rank, scal, n, mask, crank);
-          ephase ^= 1u;
-        } else if (kSolo) {
-          expand_mma(p, L, sm, w, rank, scal, n, mask, 0, p.out);
-        } else {
-          const int oc = bgmv_ochunk(p.out);
-          const int j0 = min(p.out, (int)crank * oc);
-          expand_mma(p, L, sm, w, rank, scal, n, mask, j0, min(p.out, j0 + oc));
-        }
+        expand_mma(p, L, sm, w, rank, scal, n, mask, 0, p.out);
         __syncthreads();
       }
     }
@@ -1086,14 +1066,14 @@ template <int MODE>
 cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stream,
                         const char** why) {
   BgmvParams p = p_in;
-  constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink || MODE == kModeExpert);
+  constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink);
   constexpr bool kSolo = (MODE == kModeExpertSolo);
   p.kchunk = kSolo ? p.in : bgmv_kchunk(p.in);
   bgmv_pick_stages(p.kchunk, p.S, p.R, kSolo ? kSoloRingBudget : kRingBudget, &p.kb, &p.nst);
-  const int npref = (MODE == kModeExpert || kSolo) ? p.num_experts : p.slots;
+  const int npref = kSolo ? p.num_experts : p.slots;
   const BgmvLayout L0 = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst, 0);
   const int ex_bytes = bgmv_ex_stage_bytes(p.out, p.R);
-  p.ex_stage = ((MODE == kModeFused || MODE == kModeExpert) &&
+  p.ex_stage = (MODE == kModeFused &&
                 ex_bytes <= max(p.nst * L0.stage_bytes, kExStageMax))
                    ? 1
                    : 0;
@@ -1189,7 +1169,6 @@ cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream
     case kModeExpand: return launch_mode<kModeExpand>(p, max_items, stream, why);
     case kModeEmbed: return launch_mode<kModeEmbed>(p, max_items, stream, why);
     case kModeGather: return launch_mode<kModeGather>(p, max_items, stream, why);
-    case kModeExpert: return launch_mode<kModeExpert>(p, max_items, stream, why);
     case kModeExpertSolo: return launch_mode<kModeExpertSolo>(p, max_items, stream, why);
     default: return cudaErrorInvalidValue;
   }

@@ -34,11 +34,10 @@ enum BgmvMode : int {
   kModeExpand = 2,  // expand only, h read from global
   kModeEmbed = 3,   // gather + expand (apply_embedding)
   kModeGather = 4,  // gather only (gather_shrink)
-  kModeExpert = 5,  // MoE fold (shrink + expand per (expert chunk, slot)), one cluster per chunk
-  kModeExpertSolo = 6,  // MoE fold, one CTA per (expert, slot) pair: shrink over all of in
+  kModeExpertSolo = 6,  // MoE fold: one CTA per expert chunk, shrink over all of in
 };
 
-// Ring budget of the one-CTA-per-pair MoE fold (two CTAs per SM).
+// Ring budget of the one-CTA-per-chunk MoE fold (two CTAs per SM).
 constexpr int kSoloRingBudget = 80 * 1024;
 
 struct BgmvParams {
@@ -125,8 +124,7 @@ __host__ __device__ inline BgmvLayout bgmv_layout(int mode, int npref, int S, in
   L.misc_off = off;
   off += round_up_i(kMiscInts * 4, 128);
   L.ring_off = off;
-  const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpert ||
-                     mode == kModeExpertSolo);
+  const bool ring = (mode == kModeFused || mode == kModeShrink || mode == kModeExpertSolo);
   if (ring) off += round_up_i(max(nst * L.stage_bytes, ring_min), 128);
   L.hpart_off = off;
   if (ring) off += 2 * kTT * L.srp * 4;
