@@ -294,6 +294,26 @@ def capture(torch, wl, first, count, stream):
     return g
 
 
+def rank_seed0(rank):
+    """First input seed of a rank's workload sets: each replica runs its own
+    batches (ranks draw disjoint seeds)."""
+    return 10 * rank
+
+
+def reduce_max_over_ranks(torch, dist, value, device):
+    """Max of a per-rank float over the default process group: the timed
+    region of a multi-GPU run is the slowest rank's."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, world, sec):
+    """Whole-job throughput: the units all ranks processed over the (max over
+    ranks) timed seconds."""
+    return units_per_rank_step * steps * world / sec
+
+
 def time_steps(torch, wl, steps, warmup, dist=None, sampler=None):
     """Run `warmup` steps, then time exactly `steps` steps from CUDA graphs.
     Returns (seconds for the timed steps (max over ranks), wall window)."""
@@ -340,9 +360,7 @@ def time_steps(torch, wl, steps, warmup, dist=None, sampler=None):
         dist.barrier()
     sec = e0.elapsed_time(e1) / 1e3
     if dist is not None:
-        t = torch.tensor([sec], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        sec = float(t.item())
+        sec = reduce_max_over_ranks(torch, dist, sec, "cuda")
     for g in graphs.values():
         del g
     return sec, (t_wall0, t_wall1)
@@ -560,7 +578,7 @@ def main():
         L.lora_set_launch_overlap(1)
 
     name = args.workload
-    wl = Workload(name, n_sets_for(name), 10 * rank, torch, L)
+    wl = Workload(name, n_sets_for(name), rank_seed0(rank), torch, L)
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
@@ -573,7 +591,7 @@ def main():
     clocks = sampler.summary(w0, w1)
 
     ms_per_step = sec / args.steps * 1e3
-    value = wl.tokens * args.steps * world / sec
+    value = job_throughput(wl.tokens, args.steps, world, sec)
     hbm_peak, tf_peak, peak_kind = load_peaks()
     kernel_s = sec / (args.steps * wl.launches_per_step) if wl.launches_per_step == 1 else None
     step_gbs = wl.bytes / (sec / args.steps) / 1e9

@@ -116,3 +116,10 @@ def test_host_queries(lib):
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
                                   L.LORA_REGIME_BGMV) == 0
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == L.LORA_REGIME_BGMV
+
+
+def test_launch_overlap_setting_roundtrip(lib):
+    # a process-wide flag: returns the previous setting, launches nothing
+    prev = L.lora_set_launch_overlap(1)
+    assert L.lora_set_launch_overlap(0) == 1
+    assert L.lora_set_launch_overlap(prev) == 0

@@ -470,8 +470,3 @@ def test_launch_overlap_dependent_chain(regime, graph):
     assert_close(_f64(host_bits(y)), _f64(ref), "chain")
     assert all(read_flags(d.flags) == 0 for d in devs)
 
-
-def test_launch_overlap_setting_roundtrip():
-    prev = L.lora_set_launch_overlap(1)
-    assert L.lora_set_launch_overlap(0) == 1
-    assert L.lora_set_launch_overlap(prev) == 0
