@@ -24,7 +24,9 @@
  *     must be 16-byte aligned.
  *   - The caller owns every buffer.  The library never allocates device
  *     memory and keeps no state between calls except a per-device cache of
- *     kernel attributes (SM count, occupancy).
+ *     kernel attributes (SM count, occupancy), the process-wide launch
+ *     overlap setting (lora_set_launch_overlap) and the fixed scratch array of
+ *     lora_apply_linear_noalloc, which is part of the library image.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never synchronises with the host.  The launch shape
  *     depends only on the scalar arguments, so calls can be captured in a CUDA
@@ -127,10 +129,13 @@ LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const i
 
 /*
  * lora_apply_linear -- LoraBackend.apply_linear_ (shrink then expand, fused):
- * same arguments as lora_shrink + lora_expand, with h kept on chip (BGMV) or in
- * `workspace` (SGMV).  workspace must hold lora_workspace_bytes(
- * LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, regime) bytes (may be NULL
- * when that is 0).
+ * same arguments as lora_shrink + lora_expand.  BGMV: one launch, h kept on
+ * chip.  SGMV: a tensor-core shrink writes fp32 partial h (one buffer per
+ * split of the input features) into `workspace` and the expand sums them.
+ * workspace must hold lora_workspace_bytes(LORA_OP_APPLY_LINEAR, T, slots, R,
+ * num_slices, regime) bytes and be 16-byte aligned (may be NULL when that is
+ * 0); its contents need no initialisation.  Calls sharing one workspace are
+ * ordered by their stream (with the launch overlap on too).
  */
 LORA_API lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
                               const int32_t* ranks, const float* scalings,
