@@ -85,6 +85,23 @@ def test_random_linear(regime, shape, seed):
     _check_linear(p, regime, what=f"{shape}")
 
 
+LIMIT_SHAPES = [
+    # T, in, out_slices, slots, R, ranks
+    (40, 64, (8,) * 8, 3, 16, [16, 9, 1]),     # eight slices (the limit), ranks not a multiple of 4
+    (48, 96, (32,), 2, 128, [128, 72]),         # R = 128 in one slice: 8 k-steps per expand tile
+    (70, 136, (16, 24), 4, 8, [8, 0, 5, 8]),    # R = 8 (half a k-step), a rank-0 slot
+]
+
+
+@pytest.mark.parametrize("shape", LIMIT_SHAPES)
+def test_limit_shapes_bgmv(shape):
+    """The BGMV regime at its shape limits (num_slices * roundup(R, 16) = 128),
+    with ranks that end inside a group of four columns."""
+    T, n_in, outs, slots, R, ranks = shape
+    p = W.random_linear(500, T, n_in, outs, slots, R, ranks=ranks, dead_frac=0.1)
+    _check_linear(p, L.LORA_REGIME_BGMV, what=f"{shape}")
+
+
 SGMV_SHAPES = [
     # T, in, out_slices, slots, R, ranks
     (700, 256, (136, 64), 3, 16, [16, 8, 12]),       # 3+ tiles per slot, ragged chunks
