@@ -669,14 +669,11 @@ LORA_DEV void expand_step(const uint16_t* __restrict__ bs, const uint16_t* __res
 // computes their columns.
 LORA_DEV void expand_staged(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
                             const ExStage& X, int rank, float scal, int n, uint32_t rowmask,
-                            uint32_t crank) {
+                            int j0, int j1) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int g = lane >> 2;
   const int c = lane & 3;
-  const int oc = bgmv_ochunk(p.out);
-  const int j0 = min(p.out, (int)crank * oc);
-  const int j1 = min(p.out, j0 + oc);
   const int ksteps = ceil_div_i(rank, 16);
   const int ntn = ceil_div_i(n, 8);
   const bool one = ksteps <= 1;
@@ -720,13 +717,11 @@ LORA_DEV void expand_staged(const BgmvParams& p, const BgmvLayout& L, const Smem
 // contiguous bytes of a row).  Every thread must call it after its
 // expand_staged.
 LORA_DEV void write_back_staged(const BgmvParams& p, const Smem& sm, const ExStage& X, int n,
-                                uint32_t rowmask, uint32_t crank) {
+                                uint32_t rowmask, int j0, int j1) {
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int oc = bgmv_ochunk(p.out);
-  const int j0 = min(p.out, (int)crank * oc);
-  const int cpr = (min(p.out, j0 + oc) - j0) >> 3;   // 16-byte chunks per row
+  const int cpr = (j1 - j0) >> 3;   // 16-byte chunks per row
   const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
   for (int t = warp; t < n; t += kBgmvThreads / 32) {
     if (!((live >> t) & 1u)) continue;
@@ -734,6 +729,43 @@ LORA_DEV void write_back_staged(const BgmvParams& p, const Smem& sm, const ExSta
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.y) +
                                           (size_t)sm.tok[t] * p.out + j0);
     for (int ch = lane; ch < cpr; ch += 32) dst[ch] = src[ch];
+  }
+}
+
+// Expand of one MoE group on one CTA over every output column, in chunks of
+// p.ex_cw columns: the pair's B rows and the group's y rows over a chunk are
+// staged through the (idle) ring by 16-byte cp.async copies, then updated by
+// expand_staged and written back.  Every thread must call it.
+LORA_DEV void expand_chunked(const BgmvParams& p, const BgmvLayout& L, const Smem& sm, int w,
+                             int rank, float scal, int n, uint32_t rowmask) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int cw = p.ex_cw;
+  ExStage X;
+  X.bs = sm.ring;
+  X.ys = sm.ring + round_up_i(cw * p.R * 2, 128);
+  X.ystride = cw * 2 + 16;
+  const uint32_t live = (n >= 32 ? 0xffffffffu : ((1u << n) - 1u)) & rowmask;
+  const uint16_t* bg = reinterpret_cast<const uint16_t*>(p.b) + (size_t)w * p.out * p.R;
+  const uint16_t* yg = reinterpret_cast<const uint16_t*>(p.y);
+  for (int j0 = 0; j0 < p.out; j0 += cw) {
+    const int j1 = min(p.out, j0 + cw);
+    const int bchunks = (j1 - j0) * p.R / 8;   // B rows [j0, j1) are contiguous
+    for (int i = threadIdx.x; i < bchunks; i += kBgmvThreads)
+      cp_async16(smem_u32(X.bs) + i * 16, bg + (size_t)j0 * p.R + i * 8);
+    const int ypr = (j1 - j0) / 8;             // 16-byte chunks of a y row
+    for (int t = warp; t < n; t += kBgmvThreads / 32) {
+      if (!((live >> t) & 1u)) continue;
+      const uint16_t* src = yg + (size_t)sm.tok[t] * p.out + j0;
+      const uint32_t dst = smem_u32(X.ys + t * X.ystride);
+      for (int c = lane; c < ypr; c += 32) cp_async16(dst + c * 16, src + c * 8);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    expand_staged(p, L, sm, X, rank, scal, n, rowmask, j0, j1);
+    write_back_staged(p, sm, X, n, rowmask, j0, j1);
+    __syncthreads();   // the ring is refilled for the next chunk
   }
 }
 
@@ -751,16 +783,19 @@ LORA_DEV bool wait_staged(uint64_t* bar, uint32_t parity) {
 LORA_DEV void expand_after_stage(const BgmvParams& p, const BgmvLayout& L, const Smem& sm,
                                  const ExStage& X, uint64_t* bar, uint32_t parity, int rank,
                                  float scal, int n, uint32_t rowmask, uint32_t crank) {
+  const int oc = bgmv_ochunk(p.out);
+  const int j0 = min(p.out, (int)crank * oc);
+  const int j1 = min(p.out, j0 + oc);
   const bool ok = wait_staged(bar, parity);
   if (ok) {
-    expand_staged(p, L, sm, X, rank, scal, n, rowmask, crank);
+    expand_staged(p, L, sm, X, rank, scal, n, rowmask, j0, j1);
   } else {
     if ((threadIdx.x & 31) == 0) raise_flag(p.flags, LORA_FLAG_TIMEOUT);
     wait_staged(bar, parity);
   }
   // the rows are stored only when every warp saw its copies land
   if (__syncthreads_or(ok ? 0 : 1) == 0) {
-    write_back_staged(p, sm, X, n, rowmask, crank);
+    write_back_staged(p, sm, X, n, rowmask, j0, j1);
   }
 }
 
@@ -1036,7 +1071,10 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         produce_h<kFromLocal>(p, L, sm, hp, w, rank, n, mask, true, false, 0);
         hpar ^= 1;
         __syncthreads();
-        expand_mma(p, L, sm, w, rank, scal, n, mask, 0, p.out);
+        if (p.ex_cw > 0)
+          expand_chunked(p, L, sm, w, rank, scal, n, mask);
+        else
+          expand_mma(p, L, sm, w, rank, scal, n, mask, 0, p.out);
         __syncthreads();
       }
     }
@@ -1078,6 +1116,14 @@ cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stre
                    ? 1
                    : 0;
   const BgmvLayout L = bgmv_layout(MODE, npref, p.S, p.R, p.kb, p.nst, p.ex_stage ? ex_bytes : 0);
+  // MoE fold: widest column chunk (a multiple of 64, at most 512) whose B rows
+  // and kTT y rows fit the ring, or 0 (expand straight from global memory)
+  p.ex_cw = 0;
+  if (kSolo) {
+    const int ring = p.nst * L.stage_bytes;
+    for (int cw = 512; cw >= 64 && p.ex_cw == 0; cw -= 64)
+      if (round_up_i(cw * p.R * 2, 128) + kTT * (cw * 2 + 16) <= ring) p.ex_cw = cw;
+  }
   // Wide stage rows (1 KB) go as one bulk copy each; narrower ones as 16-byte
   // cp.async copies, which land sooner for small rounds.
   p.bulk_stage = (p.kb >= 512 && (kClustered || kSolo)) ? 1 : 0;

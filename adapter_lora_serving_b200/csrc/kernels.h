@@ -68,6 +68,7 @@ struct BgmvParams {
   int nst;        // stages in the ring (1 or 2)
   int ex_stage;   // 1: the expand operands of an item fit the ring and are staged there
   int bulk_stage; // 1: shrink stages are staged by bulk copies, 0: by cp.async
+  int ex_cw;      // MoE fold: output columns per staged expand chunk (0: unstaged)
   int slice_off[LORA_MAX_SLICES + 1];
 };
 
