@@ -508,24 +508,39 @@ def time_oracle(name, prob, budget_s=12.0, min_s=10.0):
 # Profiles: DRAM traffic of the dominant kernel from a committed ncu summary
 # ---------------------------------------------------------------------------
 
-def source_digest():
+# Sources each kernel is built from: stored DRAM counters stay valid while
+# these files are unchanged.
+KERNEL_SOURCES = {
+    "bgmv_kernel": ["bgmv.cu", "common.cuh", "kernels.h"],
+    "sgmv_expand_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
+    "sgmv_shrink_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
+}
+
+
+def source_digest(kernel):
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "adapter_lora_serving_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "adapter_lora_serving_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def measured_traffic(name):
+    """DRAM bytes per launch of the workload's dominant kernel from one ncu
+    capture (profiles/traffic.json), or None once that kernel's sources differ
+    from the ones the capture was taken at."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(name)
     except (OSError, ValueError):
         return None, None
-    if not rec or rec.get("source_digest") != source_digest():
-        return None, rec.get("kernel") if rec else None
-    return rec.get("dram_bytes_per_launch"), rec.get("kernel")
+    if not rec:
+        return None, None
+    kernel = rec.get("kernel")
+    if kernel not in KERNEL_SOURCES or rec.get("source_digest") != source_digest(kernel):
+        return None, kernel
+    return rec.get("dram_bytes_per_launch"), kernel
 
 
 def load_peaks():
