@@ -102,6 +102,14 @@ def test_limit_shapes_bgmv(shape):
     _check_linear(p, L.LORA_REGIME_BGMV, what=f"{shape}")
 
 
+@pytest.mark.parametrize("regime", REGIMES)
+def test_max_slots(regime):
+    """LORA_MAX_SLOTS slots (the planner's largest prefix and item caches),
+    most of them empty, a few hundred tokens spread over the rest."""
+    p = W.random_linear(600, 300, 64, (16, 32), 4096, 16, dead_frac=0.1)
+    _check_linear(p, regime, what="4096 slots")
+
+
 SGMV_SHAPES = [
     # T, in, out_slices, slots, R, ranks
     (700, 256, (136, 64), 3, 16, [16, 8, 12]),       # 3+ tiles per slot, ragged chunks
