@@ -799,6 +799,14 @@ LORA_DEV void expand_after_stage(const BgmvParams& p, const BgmvLayout& L, const
   }
 }
 
+// k-th work item of group g of ng.  Linear targets: passes over the groups
+// alternate in direction, so the groups that drew the first (in slot order,
+// under a skewed slot load the largest) items of a pass draw the last of the
+// next one.  MoE chunks: round robin (measured better there).
+LORA_DEV int item_of(bool snake, int k, int g, int ng) {
+  return k * ng + ((snake && (k & 1)) ? (ng - 1 - g) : g);
+}
+
 }  // namespace
 
 template <int MODE>
@@ -888,7 +896,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       const int i0 = sm.prefix[sl], i1 = sm.prefix[sl + 1];
       if (i1 <= i0) continue;
       for (int k = 0; k < kItemCache; ++k) {
-        const int item = (int)group + k * (int)ngroups;
+        const int item = item_of(true, k, (int)group, (int)ngroups);
         if (item < i0 || item >= i1 || item >= total) continue;
         const int p0 = p.slot_indptr[sl] + (item - i0) * kTT;
         sm.sub_s[k] = sl;
@@ -911,7 +919,8 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
 
   int hpar = 0;
   int iter = 0;
-  for (int item = (int)group; item < total; item += (int)ngroups, ++iter) {
+  for (int item = (int)group; item < total;
+       ++iter, item = item_of(!kMoE, iter, (int)group, (int)ngroups)) {
     if (!kMoE) {
       // ---- linear / embedding item: (slot, tile of kTT positions) ----
       int s, p0, n, rank;
