@@ -169,7 +169,7 @@ lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* r
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
-      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+      return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);
     const char* why = nullptr;
     cudaError_t err = lora::sgmv_shrink_launch(x, a, h, ranks, token_order, slot_indptr, T,
                                                in_features, slots, R, num_slices, err_flags, s,
@@ -212,7 +212,7 @@ lora_status lora_expand(void* y, const float* h, const void* b, const int32_t* r
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
-      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+      return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);
     const char* why = nullptr;
     cudaError_t err = lora::sgmv_expand_launch(y, h, 1, nullptr, nullptr, b, ranks, scalings,
                                                token_order, slot_indptr, T, 0, slots, R,
@@ -257,7 +257,7 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
-      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+      return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);
     const size_t need = lora::sgmv_workspace_bytes(T, R, num_slices);
     if (workspace == nullptr || workspace_bytes < need)
       return fail(LORA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", op, need,
@@ -345,7 +345,7 @@ lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
-      return fail(LORA_ERR_UNSUPPORTED, "%s: SGMV regime needs num_slices*R <= 256 and R <= 64", op);
+      return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);
     const char* why = nullptr;
     cudaError_t err = lora::sgmv_expand_launch(y, nullptr, 1, ids, a, b, ranks, scalings,
                                                token_order, slot_indptr, T, vocab, slots, R,

@@ -12,6 +12,9 @@ constexpr int kSgmvTileM = 128;  // positions (tokens) per work item
 
 // Shapes the SGMV kernels take: R in {16, 32, 64}, num_slices * R <= 128.
 bool sgmv_supported(int S, int R);
+// The same rule as text, for error messages.
+constexpr const char* kSgmvShapeRule =
+    "the SGMV regime needs R in {16, 32, 64} and num_slices * R <= 128";
 // Workspace of lora_apply_linear in this regime (partial h buffers).
 size_t sgmv_workspace_bytes(int T, int R, int S);
 // Splits of the input features the shrink uses for these shapes.

@@ -294,10 +294,10 @@ def capture(torch, wl, first, count, stream):
     return g
 
 
-def rank_seed0(rank):
-    """First input seed of a rank's workload sets: each replica runs its own
-    batches (ranks draw disjoint seeds)."""
-    return 10 * rank
+def rank_seed0(rank, n_sets):
+    """First input seed of a rank's workload sets: rank r draws seeds
+    [r * n_sets, (r + 1) * n_sets), so every replica runs its own batches."""
+    return rank * n_sets
 
 
 def reduce_max_over_ranks(torch, dist, value, device):
@@ -314,43 +314,65 @@ def job_throughput(units_per_rank_step, steps, world, sec):
     return units_per_rank_step * steps * world / sec
 
 
-def time_steps(torch, wl, steps, warmup, dist=None, sampler=None):
-    """Run `warmup` steps, then time exactly `steps` steps from CUDA graphs.
-    Returns (seconds for the timed steps (max over ranks), wall window)."""
+def graph_counts(total, inner):
+    """Step counts of the graphs that run `total` steps in chunks of `inner`."""
+    out = []
+    if total >= inner:
+        out.append(inner)
+    if total % inner:
+        out.append(total % inner)
+    return out
+
+
+def time_steps(torch, wl, steps, warmup, dist=None, sampler=None, load_s=0.0):
+    """Run `warmup` steps, then time exactly `steps` steps replayed from CUDA
+    graphs.  Every graph the timed region replays is captured (and replayed
+    once) before the start event, and a short device-side delay is queued
+    ahead of that event so that the host's graph submissions are not timed.
+    With `load_s` > 0 the step is also replayed untimed for about that many
+    seconds just before the timed region while `sampler` records the clocks.
+    Returns (seconds for the timed steps (max over ranks), clock window)."""
     stream = torch.cuda.Stream()
     nset = len(wl.sets)
     # steps per graph: a whole number of rotations, so no set is reused early
     per = 256 if wl.tokens < 1024 else 16
     inner = nset * max(1, per // nset)
-    inner = max(1, min(steps, inner))
+    warm = max(warmup, 3)
     # eager warm-up call (sets kernel attributes before any capture)
     with torch.cuda.stream(stream):
         wl.step(0)
     torch.cuda.synchronize()
     graphs = {}
-
-    def graph_for(count):
-        if count not in graphs:
-            graphs[count] = capture(torch, wl, 0, count, stream)
-        return graphs[count]
+    for c in sorted(set(graph_counts(steps, inner) + graph_counts(warm, inner) + [inner])):
+        graphs[c] = capture(torch, wl, 0, c, stream)
 
     def run(total):
         done = 0
         while done < total:
             c = min(inner, total - done)
-            graph_for(c).replay()
+            graphs[c].replay()
             done += c
 
     with torch.cuda.stream(stream):
-        run(max(warmup, 3))
+        for g in graphs.values():      # every graph runs once before timing
+            g.replay()
+        run(warm)
+    torch.cuda.synchronize()
+    t_load0 = time.time()
+    if load_s > 0:
+        with torch.cuda.stream(stream):
+            t_end = time.time() + load_s
+            while time.time() < t_end:
+                graphs[inner].replay()
+                torch.cuda.synchronize()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    t_wall0 = time.time()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        torch.cuda._sleep(200000)      # keeps the device busy while the graphs are queued
         e0.record(stream)
         run(steps)
         e1.record(stream)
@@ -361,9 +383,8 @@ def time_steps(torch, wl, steps, warmup, dist=None, sampler=None):
     sec = e0.elapsed_time(e1) / 1e3
     if dist is not None:
         sec = reduce_max_over_ranks(torch, dist, sec, "cuda")
-    for g in graphs.values():
-        del g
-    return sec, (t_wall0, t_wall1)
+    graphs.clear()
+    return sec, (t_load0, t_wall1)
 
 
 def time_e2e(torch, wl, steps):
@@ -568,6 +589,9 @@ def main():
                     help="launch each step's kernel only after the previous one has finished")
     ap.add_argument("--profile", action="store_true",
                     help="timed steps only (no e2e, CPU baseline or table): for ncu captures")
+    ap.add_argument("--clock-window", type=float, default=0.4,
+                    help="seconds of untimed replay of the step, under the clock sampler, "
+                         "directly before the timed steps")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -593,7 +617,8 @@ def main():
         L.lora_set_launch_overlap(1)
 
     name = args.workload
-    wl = Workload(name, n_sets_for(name), rank_seed0(rank), torch, L)
+    nset = n_sets_for(name)
+    wl = Workload(name, nset, rank_seed0(rank, nset), torch, L)
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
@@ -601,9 +626,11 @@ def main():
     sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.2)
-    sec, (w0, w1) = time_steps(torch, wl, args.steps, args.warmup, dist)
+    sec, (w0, w1) = time_steps(torch, wl, args.steps, args.warmup, dist, load_s=args.clock_window)
     sampler.stop()
     clocks = sampler.summary(w0, w1)
+    clocks["window"] = (f"nvidia-smi every 50 ms over an untimed {args.clock_window:.1f} s replay "
+                        f"of the same step directly before the timed steps, and the timed steps")
 
     ms_per_step = sec / args.steps * 1e3
     value = job_throughput(wl.tokens, args.steps, world, sec)
@@ -629,7 +656,9 @@ def main():
                       "parallelism": f"replicas x{world} (independent batches, no collective)",
                       "l2": f"inputs rotate over {len(wl.sets)} independent sets "
                             f"({len(wl.sets) * wl.set_bytes / 1e6:.0f} MB > 2x L2)",
-                      "timing": "CUDA-graph replay, CUDA events on the launching stream",
+                      "timing": "CUDA-graph replay (every graph captured and replayed once "
+                                "before the start event; a device-side delay queued ahead of "
+                                "it), CUDA events on the launching stream",
                       "launch_overlap": "off" if args.no_overlap else
                       "programmatic dependent launch between consecutive steps"},
            "roofline": roofline, "clocks": clocks,

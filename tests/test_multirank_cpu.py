@@ -27,8 +27,12 @@ def _worker(rank, world, port, out):
                             world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         sec = bench.reduce_max_over_ranks(torch, dist, 0.25 * (rank + 1), "cpu")
-        seeds = [bench.rank_seed0(rank) + i for i in range(3)]
-        # every rank contributes its seeds; the union must have no repeats
+        # every rank contributes the seeds of each workload's rotating input
+        # sets (as many as bench.py draws); the union must have no repeats
+        seeds = {}
+        for name in bench.W.WORKLOADS:
+            n = bench.n_sets_for(name)
+            seeds[name] = [bench.rank_seed0(rank, n) + i for i in range(n)]
         gathered = [None] * world
         dist.all_gather_object(gathered, seeds)
         out.put((rank, sec, gathered))
@@ -50,8 +54,9 @@ def test_two_gloo_ranks_max_time_and_disjoint_seeds():
         assert p.exitcode == 0
     for rank, sec, gathered in res:
         assert sec == pytest.approx(0.5)          # the slower rank's seconds
-        flat = [s for seeds in gathered for s in seeds]
-        assert len(flat) == len(set(flat))        # independent batches per rank
+        for name in gathered[0]:
+            flat = [s for seeds in gathered for s in seeds[name]]
+            assert len(flat) == len(set(flat)), name   # independent batches per rank
 
 
 def test_job_throughput_counts_every_rank():
