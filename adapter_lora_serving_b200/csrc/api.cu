@@ -91,12 +91,25 @@ bool bgmv_fits(int S, int R) { return S * lora::round_up_i(R, 16) <= lora::kMaxS
 
 int resolve(int regime, int op, int T, int slots, int R, int S, int in_features = 1 << 30) {
   if (regime == LORA_REGIME_BGMV || regime == LORA_REGIME_SGMV) return regime;
+  if (regime == LORA_REGIME_BGMV_SPLIT)
+    return op == LORA_OP_APPLY_LINEAR ? LORA_REGIME_BGMV_SPLIT : LORA_REGIME_BGMV;
   const bool needs_shrink = (op == LORA_OP_SHRINK || op == LORA_OP_APPLY_LINEAR);
   // Many tokens per slot on average: tensor-core tiles over slot segments.
   if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024 &&
       (!needs_shrink || in_features >= 64))
     return LORA_REGIME_SGMV;
   return LORA_REGIME_BGMV;
+}
+
+// Workspace bytes lora_apply_linear needs in regime `reg` (0: none).  SGMV:
+// the counter header (which it leaves alone), then the partial h buffers of
+// the split shrink.  BGMV_SPLIT: its counters and partials.  BGMV: none.
+size_t apply_linear_need(int reg, int T, int in_features, int slots, int R, int S, int out) {
+  if (T <= 0 || R <= 0 || S <= 0) return 0;
+  if (reg == LORA_REGIME_SGMV) return lora::kWsCounterBytes + lora::sgmv_workspace_bytes(T, R, S);
+  if (reg == LORA_REGIME_BGMV_SPLIT && lora::split_eligible(T, in_features, slots, R, S, out))
+    return lora::split_workspace_bytes(T, slots, R, S);
+  return 0;
 }
 
 int linear_items_bound(int T, int slots, int tile) {
@@ -109,6 +122,11 @@ int linear_items_bound(int T, int slots, int tile) {
 namespace lora {
 // Lets other entry points of the library report through lora_last_error().
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,
+                              int out) {
+  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, S, in_features);
+  return apply_linear_need(reg, T, in_features, slots, R, S, out);
+}
 }  // namespace lora
 
 extern "C" {
@@ -138,6 +156,7 @@ int32_t lora_resolve_regime(int32_t op, int32_t T, int32_t slots, int32_t R, int
 int32_t lora_plan_tile(int32_t op, int32_t regime) {
   if (op == LORA_OP_EXPERT_APPLY) return lora::kTT;
   if (regime == LORA_REGIME_SGMV) return lora::kSgmvTileM;
+  if (op == LORA_OP_APPLY_LINEAR) return lora::kFusedTile;
   return lora::kTT;
 }
 
@@ -145,9 +164,12 @@ size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R, int
                             int32_t regime) {
   if (op != LORA_OP_APPLY_LINEAR || T <= 0 || R <= 0 || num_slices <= 0) return 0;
   const int reg = resolve(regime, op, T, slots, R, num_slices);
-  if (reg != LORA_REGIME_SGMV) return 0;
-  return lora::sgmv_workspace_bytes(T, R, num_slices);
+  // in_features and out are not known here: size for the largest the split
+  // kernel takes (it refuses larger ones)
+  return apply_linear_need(reg, T, lora::kSpMaxIn, slots, R, num_slices, lora::kSpMaxOut);
 }
+
+uint64_t lora_set_wait_limit_ns(uint64_t ns) { return lora::set_wait_limit_ns(ns); }
 
 lora_status lora_shrink(const void* x, float* h, const void* a, const int32_t* ranks,
                         const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
@@ -258,13 +280,13 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
       return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);
-    const size_t need = lora::sgmv_workspace_bytes(T, R, num_slices);
+    const size_t need = apply_linear_need(reg, T, in_features, slots, R, num_slices, out);
     if (workspace == nullptr || workspace_bytes < need)
       return fail(LORA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", op, need,
                   workspace == nullptr ? (size_t)0 : workspace_bytes);
     if (!aligned16(workspace))
       return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
-    float* hws = static_cast<float*>(workspace);
+    float* hws = reinterpret_cast<float*>(static_cast<char*>(workspace) + lora::kWsCounterBytes);
     const char* why = nullptr;
     const int ks = lora::sgmv_shrink_splits(T, slots, in_features);
     cudaError_t err = lora::sgmv_shrink_launch(x, a, hws, ranks, token_order, slot_indptr, T,
@@ -280,12 +302,41 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
   if (!bgmv_fits(num_slices, R))
     return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
                 num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
+  if (reg == LORA_REGIME_BGMV_SPLIT) {
+    // the split kernel: every SM shares the work, h partials through the workspace
+    if (!lora::split_eligible(T, in_features, slots, R, num_slices, out))
+      return fail(LORA_ERR_UNSUPPORTED,
+                  "%s: BGMV_SPLIT takes T <= %d, slots <= %d, at most %d work items, "
+                  "in_features <= %d, out <= %d and num_slices*roundup(R,16) <= %d",
+                  op, lora::kSpMaxT, lora::kSpMaxSlots, lora::kSpMaxItems, lora::kSpMaxIn,
+                  lora::kSpMaxOut, lora::kMaxSRp);
+    const size_t need = lora::split_workspace_bytes(T, slots, R, num_slices);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(LORA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", op, need,
+                  workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned16(workspace))
+      return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
+    lora::SplitParams q = {};
+    q.x = x; q.y = y; q.a = a; q.b = b; q.ranks = ranks; q.scalings = scalings;
+    q.token_order = token_order; q.slot_indptr = slot_indptr; q.flags = err_flags;
+    const int cap = lora::split_item_cap(T, slots);
+    q.cnt = static_cast<uint32_t*>(workspace);
+    q.cons = q.cnt + cap;
+    q.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lora::kWsCounterBytes);
+    q.T = T; q.in = in_features; q.slots = slots; q.R = R; q.S = num_slices; q.out = out;
+    q.item_cap = cap;
+    for (int i = 0; i <= LORA_MAX_SLICES; ++i) q.slice_off[i] = p.slice_off[i];
+    const char* why = nullptr;
+    cudaError_t err = lora::split_launch(q, s, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
   p.x = x; p.y = y; p.a = a; p.b = b; p.ranks = ranks; p.scalings = scalings;
   p.token_order = token_order; p.slot_indptr = slot_indptr; p.flags = err_flags; p.T = T;
   p.in = in_features; p.slots = slots; p.R = R; p.S = num_slices; p.out = out;
   const char* why = nullptr;
-  cudaError_t err = lora::bgmv_launch(lora::kModeFused, p, linear_items_bound(T, slots, lora::kTT),
-                                      s, &why);
+  cudaError_t err = lora::bgmv_launch(lora::kModeFused, p,
+                                      linear_items_bound(T, slots, lora::kFusedTile), s, &why);
   if (err != cudaSuccess) return cuda_fail(err, op, why);
   return ok();
 }

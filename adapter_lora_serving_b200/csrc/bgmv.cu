@@ -22,6 +22,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "expand_tile.cuh"
 #include "kernels.h"
 
 namespace lora {
@@ -574,92 +575,6 @@ LORA_DEV void prefetch_expand(const BgmvParams& p, const Smem& sm, int w, int n,
                      (uint32_t)(cols * 2));
 }
 
-// Zero masks of the bf16 B elements k0..k0+3 at or past the rank (as
-// mask_rank4): .x covers (k0, k0+1), .y covers (k0+2, k0+3).
-LORA_DEV uint2 rank_mask4(int k0, int rank) {
-  return make_uint2((k0 < rank ? 0xffffu : 0u) | (k0 + 1 < rank ? 0xffff0000u : 0u),
-                    (k0 + 2 < rank ? 0xffffu : 0u) | (k0 + 3 < rank ? 0xffff0000u : 0u));
-}
-
-constexpr int kExGroup = 4;   // 16-column tiles a warp expands per step
-
-// One step of the staged expand: kExGroup 16-column tiles (columns jt + 128 q)
-// of one slice and one 8-token tile.  All shared-memory loads of the step are
-// issued before any MMA or store (the B copy, the h tiles and the y rows do
-// not overlap), so the tiles' latencies overlap.  ks0 < ksteps k-steps of 16
-// ranks; hh/hl are the h fragments of k-step 0 when kOneStep.
-template <bool kOneStep>
-LORA_DEV void expand_step(const uint16_t* __restrict__ bs, const uint16_t* __restrict__ hhi,
-                          const uint16_t* __restrict__ hlo, uint8_t* __restrict__ yt, int ystride,
-                          int R, int hrow, int ksteps, int rank, uint2 m0, uint2 hh, uint2 hl,
-                          int jt, int ls1, int g, int c, uint32_t lv, float scal) {
-  int jl[kExGroup];
-  bool ok[kExGroup];
-  float d[kExGroup][4];
-  uint32_t yo[kExGroup][2];
-#pragma unroll
-  for (int q = 0; q < kExGroup; ++q) {
-    jl[q] = jt + q * (kBgmvThreads / 2) + 2 * g;
-    ok[q] = jl[q] < ls1;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) d[q][k] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
-      yo[q][e] = (ok[q] && ((lv >> e) & 1u))
-                     ? *reinterpret_cast<const uint32_t*>(yt + e * ystride + jl[q] * 2)
-                     : 0u;
-  }
-  if (kOneStep) {
-    uint2 b0[kExGroup], b1[kExGroup];
-#pragma unroll
-    for (int q = 0; q < kExGroup; ++q) {
-      b0[q] = b1[q] = make_uint2(0u, 0u);
-      if (ok[q]) {
-        b0[q] = *reinterpret_cast<const uint2*>(bs + (size_t)jl[q] * R + 4 * c);
-        b1[q] = *reinterpret_cast<const uint2*>(bs + (size_t)(jl[q] + 1) * R + 4 * c);
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < kExGroup; ++q) {
-      const uint2 x0 = make_uint2(b0[q].x & m0.x, b0[q].y & m0.y);
-      const uint2 x1 = make_uint2(b1[q].x & m0.x, b1[q].y & m0.y);
-      mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, hh.x, hh.y);
-      mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, hl.x, hl.y);
-    }
-  } else {
-#pragma unroll 1
-    for (int ks = 0; ks < ksteps; ++ks) {
-      const int k0 = ks * 16 + 4 * c;
-      const uint2 mk = rank_mask4(k0, rank);
-      const uint2 h1 = *reinterpret_cast<const uint2*>(hhi + hrow + k0);
-      const uint2 h2 = *reinterpret_cast<const uint2*>(hlo + hrow + k0);
-#pragma unroll
-      for (int q = 0; q < kExGroup; ++q) {
-        uint2 x0 = make_uint2(0u, 0u), x1 = make_uint2(0u, 0u);
-        if (ok[q] && k0 < R) {
-          x0 = *reinterpret_cast<const uint2*>(bs + (size_t)jl[q] * R + k0);
-          x1 = *reinterpret_cast<const uint2*>(bs + (size_t)(jl[q] + 1) * R + k0);
-        }
-        x0 = make_uint2(x0.x & mk.x, x0.y & mk.y);
-        x1 = make_uint2(x1.x & mk.x, x1.y & mk.y);
-        mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, h1.x, h1.y);
-        mma_bf16_16816(d[q], x0.x, x1.x, x0.y, x1.y, h2.x, h2.y);
-      }
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < kExGroup; ++q) {
-    if (!ok[q]) continue;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      if ((lv >> e) & 1u)
-        *reinterpret_cast<uint32_t*>(yt + e * ystride + jl[q] * 2) =
-            pack_bf16x2(fmaf(scal, d[q][e], bf16_lo(yo[q][e])),
-                        fmaf(scal, d[q][2 + e], bf16_hi(yo[q][e])));
-    }
-  }
-}
-
 // Expand of a staged item with the m16n8k16 MMAs of expand_mma (same operands,
 // same order, so the same results): D[16 columns, 8 tokens] = B H^T per 16-column
 // tile of one slice, H = hi + lo.  B comes from the staged copy and y = bf16_rne(
@@ -880,7 +795,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
                                       kTT, sm.prefix, sm.scratch, p.flags, report);
   } else {
     total = plan_linear<kBgmvThreads>(p.slot_indptr, p.ranks, kScaled ? p.scalings : nullptr,
-                                      p.slots, p.T, p.R, kTT, sm.prefix, sm.scratch, p.flags,
+                                      p.slots, p.T, p.R, p.tile, sm.prefix, sm.scratch, p.flags,
                                       report);
   }
 #pragma unroll
@@ -898,12 +813,12 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
       for (int k = 0; k < kItemCache; ++k) {
         const int item = item_of(true, k, (int)group, (int)ngroups);
         if (item < i0 || item >= i1 || item >= total) continue;
-        const int p0 = p.slot_indptr[sl] + (item - i0) * kTT;
+        const int p0 = p.slot_indptr[sl] + (item - i0) * p.tile;
         sm.sub_s[k] = sl;
         sm.sub_s[kItemCache + k] = p.ranks[sl];
         sm.sub_p[k] = p0;
         sm.sub_p[kItemCache + k] = kScaled ? __float_as_int(p.scalings[sl]) : 0;
-        sm.sub_cnt[k] = max(0, min(kTT, p.slot_indptr[sl + 1] - p0));
+        sm.sub_cnt[k] = max(0, min(p.tile, p.slot_indptr[sl + 1] - p0));
       }
     }
   }
@@ -933,8 +848,8 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(const BgmvParams 
         n = sm.sub_cnt[iter];
       } else {
         s = find_segment(sm.prefix, p.slots, item);
-        p0 = p.slot_indptr[s] + (item - sm.prefix[s]) * kTT;
-        n = max(0, min(kTT, p.slot_indptr[s + 1] - p0));
+        p0 = p.slot_indptr[s] + (item - sm.prefix[s]) * p.tile;
+        n = max(0, min(p.tile, p.slot_indptr[s + 1] - p0));
         rank = p.ranks[s];
         scal = kScaled ? p.scalings[s] : 0.f;
       }
@@ -1113,6 +1028,7 @@ template <int MODE>
 cudaError_t launch_mode(const BgmvParams& p_in, int max_items, cudaStream_t stream,
                         const char** why) {
   BgmvParams p = p_in;
+  p.tile = MODE == kModeFused ? kFusedTile : kTT;
   constexpr bool kClustered = (MODE == kModeFused || MODE == kModeShrink);
   constexpr bool kSolo = (MODE == kModeExpertSolo);
   p.kchunk = kSolo ? p.in : bgmv_kchunk(p.in);

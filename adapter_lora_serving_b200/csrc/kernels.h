@@ -17,7 +17,8 @@ namespace lora {
 // ---------------------------------------------------------------------------
 
 constexpr int kBgmvThreads = 256;
-constexpr int kTT = 32;          // tokens (sorted rows) per work item
+constexpr int kTT = 32;          // tokens (sorted rows) per work item, at most
+constexpr int kFusedTile = 32;   // positions per work item of the fused linear path
 constexpr int kGroup = 8;        // CTAs per work item (cluster size)
 constexpr int kMaxKB = 512;      // input features per pipeline stage (upper bound)
 constexpr int kRingBudget = 120 * 1024;  // shared-memory bytes for the staging ring
@@ -69,6 +70,7 @@ struct BgmvParams {
   int ex_stage;   // 1: the expand operands of an item fit the ring and are staged there
   int bulk_stage; // 1: shrink stages are staged by bulk copies, 0: by cp.async
   int ex_cw;      // MoE fold: output columns per staged expand chunk (0: unstaged)
+  int tile;       // positions per work item of the linear modes (<= kTT)
   int slice_off[LORA_MAX_SLICES + 1];
 };
 
@@ -158,6 +160,136 @@ inline void bgmv_pick_stages(int kchunk, int S, int R, int budget, int* kb, int*
 // kernel and the SGMV kernels (lora_set_launch_overlap).
 int bgmv_set_overlap(int enable);
 bool launch_overlap_enabled();
+// Process-wide limit of every bounded device wait of the split kernel
+// (lora_set_wait_limit_ns); 0 restores the default of one second.
+uint64_t set_wait_limit_ns(uint64_t ns);
+uint64_t wait_limit_ns();
+
+// ---------------------------------------------------------------------------
+// BGMV regime, split kernel (fused apply_linear with a workspace): one CTA per
+// SM.  The shrink of every work item (<= kTT tokens of one slot) is cut along
+// the input features and the expand along the output columns, both into
+// contiguous byte ranges of equal size, one range per CTA.  Shrink pieces
+// publish fp32 partial h through the workspace and count themselves on a
+// per-item counter; the expand of an item waits (bounded) for its count and
+// sums the partials in piece order.
+// ---------------------------------------------------------------------------
+
+constexpr int kSpKQ = 64;         // input features per block of the shrink split
+constexpr int kSpCQ = 64;         // output columns per block of the expand split
+constexpr int kSpMaxGrid = 256;   // CTAs of one launch at most (workspace bound)
+constexpr int kSpMaxT = 1024;     // tokens (token_order is held in shared memory)
+constexpr int kSpMaxSlots = 1024;
+constexpr int kSpMaxItems = 512;  // work items a call may plan
+constexpr int kSpMaxIn = 65536;   // keeps every byte count of the split in 32 bits
+constexpr int kSpMaxOut = 262144;
+constexpr int kSpRingMin = 64 * 1024;   // staging ring of larger shapes (two per SM no longer fit)
+// Leading bytes of an apply_linear workspace that hold the split kernel's
+// counters; the SGMV kernels use the bytes after them.
+constexpr size_t kWsCounterBytes = 4096;
+
+struct SplitParams {
+  const void* x;               // bf16 [T, in]
+  void* y;                     // bf16 [T, out]
+  const void* a;               // bf16 [slots, S*R, in]
+  const void* b;               // bf16 [slots, out, R]
+  const int* ranks;
+  const float* scalings;
+  const int* token_order;
+  const int* slot_indptr;
+  uint32_t* cnt;               // [item_cap] shrink pieces published per item
+  uint32_t* cons;              // [item_cap] expand pieces that consumed an item
+  float* part;                 // [(item_cap + kSpMaxGrid) * kTT * S * R] partial h
+  uint32_t* flags;
+  unsigned long long wait_ns;  // bounded-wait limit
+  int T, in, slots, R, S, out;
+  int item_cap;                // items planned at most (workspace capacity)
+  int ring;                    // bytes of the staging ring (split_ring_bytes)
+  int slice_off[LORA_MAX_SLICES + 1];
+};
+
+struct SplitLayout {
+  int tok_off;    // int [T]: token_order, each slot's tokens in canonical order
+  int meta_off;   // int4 [item_cap]: slot, first position, slot tokens, rank|tile|count
+  int wcum_off;   // u32 [item_cap + 1]: exclusive prefix of shrink units
+  int vcum_off;   // u32 [item_cap + 1]: exclusive prefix of expand units
+  int cand_off;   // int [kSpMaxGrid]: the shrink pieces of the current expand item
+  int wst_off;    // u32 [kSpMaxGrid + 1]: first shrink unit of every CTA
+  int vst_off;    // u32 [kSpMaxGrid + 1]: first expand unit of every CTA
+  int ctrl_off;   // int [64]: scan scratch and broadcast words
+  int xtab_off;   // int [256]: the current expand round's job and piece tables
+  int ring_off;   // staging ring: shrink rounds, then expand jobs (and their pieces' h)
+  int total;
+};
+
+__host__ __device__ inline int split_fixed_bytes(int T, int item_cap) {
+  return round_up_i(T * 4, 128) + round_up_i(item_cap * 16, 128) +
+         2 * round_up_i((item_cap + 1) * 4, 128) + kSpMaxGrid * 4 +
+         2 * round_up_i((kSpMaxGrid + 1) * 4, 128) + 64 * 4 + 256 * 4;
+}
+
+__host__ __device__ inline SplitLayout split_layout(int T, int item_cap, int ring) {
+  SplitLayout L;
+  int off = 0;
+  L.tok_off = off;
+  off += round_up_i(T * 4, 128);
+  L.meta_off = off;
+  off += round_up_i(item_cap * 16, 128);
+  L.wcum_off = off;
+  off += round_up_i((item_cap + 1) * 4, 128);
+  L.vcum_off = off;
+  off += round_up_i((item_cap + 1) * 4, 128);
+  L.cand_off = off;
+  off += kSpMaxGrid * 4;
+  L.wst_off = off;
+  off += round_up_i((kSpMaxGrid + 1) * 4, 128);
+  L.vst_off = off;
+  off += round_up_i((kSpMaxGrid + 1) * 4, 128);
+  L.ctrl_off = off;
+  off += 64 * 4;
+  L.xtab_off = off;
+  off += 256 * 4;
+  L.ring_off = off;
+  off += ring;
+  L.total = off;
+  return L;
+}
+
+// Row stride (floats) of the fp32 h rows an expand piece keeps in the ring.
+__host__ __device__ inline int split_hst(int R) { return round_up_i(R, 16); }
+
+// The staging ring: what keeps a CTA within `budget` bytes of shared memory
+// (so that two CTAs fit one SM: one of this launch and one of the next, which
+// starts early under the launch overlap), at least kSpRingMin.
+inline int split_ring_bytes(int T, int item_cap, int budget) {
+  const int r = (budget - split_fixed_bytes(T, item_cap)) & ~127;
+  return r > kSpRingMin ? r : kSpRingMin;
+}
+
+// Items a call with these shapes can plan at most: every used slot has one
+// item per kTT of its tokens.
+inline int split_item_cap(int T, int slots) {
+  const long long c = (long long)(T < slots ? T : slots) + ceil_div_i(T, kTT);
+  return (int)(c > (1 << 30) ? (1 << 30) : c);
+}
+// Whether the split kernel takes these shapes (else the cluster kernel runs).
+inline bool split_eligible(int T, int in, int slots, int R, int S, int out) {
+  return T <= kSpMaxT && slots <= kSpMaxSlots && in <= kSpMaxIn && out <= kSpMaxOut &&
+         S * round_up_i(R, 16) <= kMaxSRp && split_item_cap(T, slots) <= kSpMaxItems;
+}
+// Workspace bytes of the split kernel: counters, then the partial h of every
+// (item, CTA) piece.
+inline size_t split_workspace_bytes(int T, int slots, int R, int S) {
+  const size_t cap = (size_t)split_item_cap(T, slots);
+  return kWsCounterBytes + (cap + kSpMaxGrid) * kTT * (size_t)S * R * sizeof(float);
+}
+
+cudaError_t split_launch(const SplitParams& p, cudaStream_t stream, const char** why);
+
+// Workspace bytes lora_apply_linear needs for these shapes in `regime` (AUTO
+// resolved with the real in_features), 0 if none (api.cu).
+size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,
+                              int out);
 
 // Launchers (bgmv.cu).  Return a cudaError_t from the launch.
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,

@@ -28,6 +28,8 @@
 
 namespace lora {
 void set_last_error(const char* msg);  // api.cu
+size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,
+                              int out);  // api.cu
 }
 
 namespace {
@@ -47,8 +49,16 @@ lora_status lora_apply_linear_noalloc(const void* x, void* y, const void* a, con
                                       int32_t T, int32_t in_features, int32_t slots, int32_t R,
                                       const int32_t* out_slices, int32_t num_slices,
                                       int32_t regime, uint32_t* err_flags, void* stream) {
-  const size_t need = lora_workspace_bytes(LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, regime);
   char msg[256];
+  long long out = 0;
+  if (out_slices != nullptr && num_slices >= 1 && num_slices <= LORA_MAX_SLICES)
+    for (int i = 0; i < num_slices; ++i) out += out_slices[i];
+  // the scratch these shapes take in the regime lora_apply_linear resolves
+  // them to (argument errors are left to lora_apply_linear to report)
+  const size_t need =
+      (out > 0 && out < (1LL << 30))
+          ? lora::apply_linear_workspace(regime, T, in_features, slots, R, num_slices, (int)out)
+          : 0;
   if (need > (size_t)LORA_STATIC_SCRATCH_BYTES) {
     snprintf(msg, sizeof(msg),
              "lora_apply_linear_noalloc: these shapes need %zu bytes of scratch; the static "

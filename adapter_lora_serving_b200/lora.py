@@ -31,6 +31,7 @@ LORA_FLAG_TIMEOUT = 64
 LORA_REGIME_AUTO = 0
 LORA_REGIME_BGMV = 1
 LORA_REGIME_SGMV = 2
+LORA_REGIME_BGMV_SPLIT = 3
 
 LORA_OP_SHRINK = 0
 LORA_OP_EXPAND = 1
@@ -63,6 +64,7 @@ _SIGS = [
     ("lora_plan_linear", _I, [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
     ("lora_plan_expert", _I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
     ("lora_set_launch_overlap", _I, [_I]),
+    ("lora_set_wait_limit_ns", ctypes.c_uint64, [ctypes.c_uint64]),
     ("lora_status_string", ctypes.c_char_p, [_I]),
     ("lora_last_error", ctypes.c_char_p, []),
     ("lora_version", ctypes.c_char_p, []),
@@ -220,6 +222,12 @@ def lora_set_launch_overlap(enable):
     """Opt in or out of overlapping the fused few-tokens kernel's start with
     the preceding kernel in the stream; returns the previous setting."""
     return int(load().lora_set_launch_overlap(1 if enable else 0))
+
+
+def lora_set_wait_limit_ns(ns):
+    """Limit (ns) of the split kernel's bounded device waits; 0 = the default
+    of one second.  Returns the previous setting."""
+    return int(load().lora_set_wait_limit_ns(int(ns)))
 
 
 def lora_version():

@@ -145,7 +145,8 @@ class Workload:
         ws = self.L.lora_workspace_bytes(self.L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R,
                                          p.num_slices)
         d["ws_bytes"] = ws
-        d["ws"] = self.torch.empty(max(ws, 16) // 4, dtype=self.torch.float32,
+        # zeroed once: the library keeps its counter header zeroed between calls
+        d["ws"] = self.torch.zeros(max(ws, 16) // 4, dtype=self.torch.float32,
                                    device="cuda") if ws else None
         return d
 

@@ -25,7 +25,8 @@
  *   - The caller owns every buffer.  The library never allocates device
  *     memory and keeps no state between calls except a per-device cache of
  *     kernel attributes (SM count, occupancy), the process-wide launch
- *     overlap setting (lora_set_launch_overlap) and the fixed scratch array of
+ *     overlap and wait-limit settings (lora_set_launch_overlap,
+ *     lora_set_wait_limit_ns) and the fixed scratch array of
  *     lora_apply_linear_noalloc, which is part of the library image.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never synchronises with the host.  The launch shape
@@ -86,6 +87,8 @@ typedef enum {
 #define LORA_REGIME_AUTO 0
 #define LORA_REGIME_BGMV 1   /* few tokens per slot: thread-block-cluster kernel, h kept on chip */
 #define LORA_REGIME_SGMV 2   /* many tokens per slot: tcgen05/TMEM tiles over slot segments */
+#define LORA_REGIME_BGMV_SPLIT 3  /* few tokens per slot, the work split by bytes over every SM
+                                     (lora_apply_linear only; needs a zeroed workspace) */
 
 #define LORA_MAX_SLICES 8
 #define LORA_MAX_SLOTS 4096
@@ -129,13 +132,26 @@ LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const i
 
 /*
  * lora_apply_linear -- LoraBackend.apply_linear_ (shrink then expand, fused):
- * same arguments as lora_shrink + lora_expand.  BGMV: one launch, h kept on
- * chip.  SGMV: a tensor-core shrink writes fp32 partial h (one buffer per
- * split of the input features) into `workspace` and the expand sums them.
+ * same arguments as lora_shrink + lora_expand.
+ *   BGMV: one launch, one thread-block cluster per work item (up to 32 tokens
+ *     of one slot), h kept in distributed shared memory; no workspace.
+ *   SGMV: a tensor-core shrink writes fp32 partial h (one buffer per split of
+ *     the input features) into the workspace and the expand sums them.
+ *   BGMV_SPLIT (only when asked for): one launch over every SM; the shrink is
+ *     cut along the input features and the expand along the output columns
+ *     into equal shares, and fp32 partial h pass through the workspace (each
+ *     work item's expand waits, bounded, for its partials; lora_set_wait_limit_ns).
+ *     Shapes beyond its limits (T > 1024, slots > 1024, more than 512 work
+ *     items possible, in_features > 65536, out > 262144) return
+ *     LORA_ERR_UNSUPPORTED.
  * workspace must hold lora_workspace_bytes(LORA_OP_APPLY_LINEAR, T, slots, R,
  * num_slices, regime) bytes and be 16-byte aligned (may be NULL when that is
- * 0); its contents need no initialisation.  Calls sharing one workspace are
- * ordered by their stream (with the launch overlap on too).
+ * 0).  Its first 4096 bytes are the BGMV_SPLIT counters: a workspace that
+ * BGMV_SPLIT calls use must be ZEROED before its first use (e.g. one
+ * cudaMemsetAsync); every call leaves them zeroed again (zero them again after a
+ * call that raised LORA_FLAG_TIMEOUT).  The rest needs no initialisation.
+ * Calls sharing one workspace must be ordered (one stream, with the launch
+ * overlap on too).
  */
 LORA_API lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
                               const int32_t* ranks, const float* scalings,
@@ -273,6 +289,16 @@ LORA_API lora_status lora_plan_expert(const int32_t* expert_offsets, const int32
  * after the call.  Returns the previous setting.
  */
 LORA_API int32_t lora_set_launch_overlap(int32_t enable);
+
+/*
+ * lora_set_wait_limit_ns -- the limit of every bounded device wait of the
+ * BGMV_SPLIT kernel (an expand waiting for its item's partial h), in
+ * nanoseconds; 0 restores the default of one second.  A wait that runs out
+ * raises LORA_FLAG_TIMEOUT, skips that work item's update of y and lets the
+ * call finish.  Process-wide; takes effect for launches issued after the
+ * call.  Returns the previous setting (0 = the default).
+ */
+LORA_API uint64_t lora_set_wait_limit_ns(uint64_t ns);
 
 LORA_API const char* lora_status_string(lora_status status);
 LORA_API const char* lora_last_error(void);

@@ -61,13 +61,17 @@ class LinearDev:
         self.slot_indptr = dev_i32(p.slot_indptr)
         self.flags = flags_buf()
 
-    def apply_linear(self, regime=L.LORA_REGIME_AUTO, workspace=None, out_slices=None):
+    def apply_linear(self, regime=L.LORA_REGIME_AUTO, workspace=None, out_slices=None,
+                     use_workspace=True):
+        """lora_apply_linear with a zeroed workspace of lora_workspace_bytes (the
+        BGMV split kernel, or SGMV), or with none (use_workspace=False: the BGMV
+        cluster kernel)."""
         p = self.p
         ws_bytes = L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R,
-                                          p.num_slices, regime)
+                                          p.num_slices, regime) if use_workspace else 0
         if ws_bytes and workspace is None:
             t = torch()
-            workspace = t.empty(ws_bytes // 4 + 4, dtype=t.float32, device="cuda")
+            workspace = t.zeros(ws_bytes // 4 + 4, dtype=t.float32, device="cuda")
         L.lora_apply_linear(self.x, self.y, self.a, self.b, self.ranks, self.scalings,
                             self.token_order, self.slot_indptr, p.T, p.n_in, p.slots, p.R,
                             out_slices or p.out_slices, regime=regime, workspace=workspace,

@@ -113,9 +113,30 @@ def test_status_strings(lib):
 def test_host_queries(lib):
     assert L.lora_plan_tile(L.LORA_OP_APPLY_LINEAR, L.LORA_REGIME_BGMV) == 32
     assert L.lora_plan_tile(L.LORA_OP_EXPERT_APPLY, L.LORA_REGIME_AUTO) == 32
+    # the cluster kernel keeps h on chip
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
                                   L.LORA_REGIME_BGMV) == 0
+    # the split kernel: 4096 bytes of counters, then one fp32 partial h tile of
+    # 32 tokens x S*R per (work item, CTA) pair: at most min(T, slots) +
+    # ceil(T/32) items, 256 CTAs
+    items = min(256, 32) + 256 // 32
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
+                                  L.LORA_REGIME_BGMV_SPLIT) == \
+        4096 + (items + 256) * 32 * 3 * 16 * 4
+    # beyond its limits it takes nothing (the call is refused)
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 2000, 64, 16, 3,
+                                  L.LORA_REGIME_BGMV_SPLIT) == 0
+    # SGMV: the counter header, then up to four fp32 partial h buffers
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 8192, 16, 64, 2,
+                                  L.LORA_REGIME_SGMV) == 4096 + 4 * 8192 * 64 * 2 * 4
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == L.LORA_REGIME_BGMV
+
+
+def test_wait_limit_setting_roundtrip(lib):
+    # a process-wide setting: returns the previous value, launches nothing
+    prev = L.lora_set_wait_limit_ns(5_000_000)
+    assert L.lora_set_wait_limit_ns(0) == 5_000_000
+    assert L.lora_set_wait_limit_ns(prev) == 0
 
 
 def test_launch_overlap_setting_roundtrip(lib):
@@ -123,3 +144,13 @@ def test_launch_overlap_setting_roundtrip(lib):
     prev = L.lora_set_launch_overlap(1)
     assert L.lora_set_launch_overlap(0) == 1
     assert L.lora_set_launch_overlap(prev) == 0
+
+
+def test_split_regime_refuses_shapes_beyond_its_limits(lib):
+    # 2000 tokens is past the split kernel's token limit: refused before launch
+    ws = 1 << 20
+    assert _apply(lib, T=2000, regime=L.LORA_REGIME_BGMV_SPLIT, ws=ws, ws_bytes=1 << 30) == \
+        L.LORA_ERR_UNSUPPORTED
+    assert "BGMV_SPLIT" in lib.lora_last_error().decode()
+    # within its limits but without a workspace: refused before launch
+    assert _apply(lib, regime=L.LORA_REGIME_BGMV_SPLIT) == L.LORA_ERR_WORKSPACE

@@ -94,6 +94,16 @@ def test_expert_plan_hand_example():
     assert [list(c) for c in chunks] == g["expected_chunks"]
 
 
+def test_adapted_experts_hand_example():
+    g = _load("adapted_experts_hand.json")
+    assert O.adapted_experts(g["pair_index"], g["slots"], g["num_experts"]) == \
+        g["expected_adapted"]
+    chunks, flags = O.plan_expert(g["expert_offsets"], g["pair_index"], g["slots"],
+                                  g["num_experts"], g["rows_cap"], g["max_rows"])
+    assert [list(c) for c in chunks] == g["expected_chunks"]
+    assert flags == g["expected_flags"]
+
+
 def test_expert_fold_hand_example():
     g = _load("expert_fold_hand.json")
     args = dict(x=np.array(g["x"], float), y=np.array(g["y"], float),
@@ -415,3 +425,21 @@ def test_planted_transposed_gather_fails_closed_form():
     x1[np.arange(p.T), p.ids] = 1.0
     h_s, m_s, _ = O.shrink(x1, a, p.token_order, p.slot_indptr, p.ranks, R, 1)
     assert not np.array_equal(h_w[m_w], h_s[m_s])
+
+
+def test_planted_unsorted_adapted_list_fails_golden(monkeypatch):
+    # experts in the order the pairs are met (slot by slot), not sorted
+    g = _load("adapted_experts_hand.json")
+
+    def first_seen(pair_index, slots, num_experts):
+        pi = np.asarray(pair_index).reshape(slots, num_experts)
+        out = []
+        for s in range(slots):
+            for e in range(num_experts):
+                if pi[s, e] != -1 and e not in out:
+                    out.append(e)
+        return out
+    monkeypatch.setattr(O, "adapted_experts", first_seen)
+    chunks, _ = O.plan_expert(g["expert_offsets"], g["pair_index"], g["slots"],
+                              g["num_experts"], g["rows_cap"], g["max_rows"])
+    assert [list(c) for c in chunks] != g["expected_chunks"]

@@ -13,14 +13,50 @@ from gpu_util import (LinearDev, MoEDev, assert_close, assert_rows_bit_identical
 
 pytestmark = pytest.mark.gpu
 
-REGIMES = [pytest.param(L.LORA_REGIME_BGMV, id="bgmv"),
-           pytest.param(L.LORA_REGIME_SGMV, id="sgmv")]
+class Path:
+    """A kernel path of lora_apply_linear: the regime hint, and whether the call
+    gets the workspace lora_workspace_bytes asks for."""
+
+    def __init__(self, regime, workspace):
+        self.regime = regime
+        self.workspace = workspace
+
+    def __eq__(self, other):        # compares as its regime
+        return self.regime == (other.regime if isinstance(other, Path) else other)
+
+    def __int__(self):
+        return self.regime
+
+
+SPLIT = Path(L.LORA_REGIME_BGMV_SPLIT, True)
+CLUSTER = Path(L.LORA_REGIME_BGMV, True)
+SGMV = Path(L.LORA_REGIME_SGMV, True)
+REGIMES = [pytest.param(SPLIT, id="bgmv_split"),
+           pytest.param(CLUSTER, id="bgmv_cluster"),
+           pytest.param(SGMV, id="sgmv")]
+
+
+def _apply(d, path, **kw):
+    path = path if isinstance(path, Path) else Path(path, True)
+    d.apply_linear(path.regime, use_workspace=path.workspace, **kw)
+
+
+def split_takes(p):
+    """The shapes the BGMV_SPLIT kernel takes (it refuses the others)."""
+    items = min(p.T, p.slots) + -(-p.T // 32)
+    return (p.T <= 1024 and p.slots <= 1024 and items <= 512 and p.n_in <= 65536 and
+            p.out <= 262144 and p.num_slices * (-(-p.R // 16) * 16) <= 128)
 
 
 def _skip_unsupported(p, regime, shrink=True):
     """The SGMV kernels take R in {16, 32, 64}, num_slices * R <= 128 and (for the
-    shrink) in_features >= 64; other shapes are the BGMV regime's."""
-    if regime != L.LORA_REGIME_SGMV:
+    shrink) in_features >= 64; the BGMV_SPLIT kernel the shapes of split_takes;
+    other shapes are the BGMV regime's."""
+    if int(regime) == L.LORA_REGIME_BGMV_SPLIT:
+        if not split_takes(p):
+            pytest.skip("shape outside the BGMV_SPLIT kernel's limits")
+        return
+    if int(regime) != L.LORA_REGIME_SGMV:
         return
     if p.R not in (16, 32, 64) or p.num_slices * p.R > 128:
         pytest.skip("shape outside the SGMV regime")
@@ -42,7 +78,7 @@ def _oracle_linear(p, y_bits=None, token_order=None):
 def _check_linear(p, regime, y_bits=None, what=""):
     _skip_unsupported(p, regime)
     d = LinearDev(p, y_bits)
-    d.apply_linear(regime)
+    _apply(d, regime)
     y_in = p.y if y_bits is None else y_bits
     out = host_bits(d.y)
     y_ref, touched, flags = _oracle_linear(p, y_in)
@@ -155,7 +191,7 @@ def test_noops_bit_exact_and_poison_ignored(regime):
         b[s, :, r:] = 0x7FC0
     p2 = W.LinearProblem(**{**p.__dict__, "a": a, "b": b})
     d = LinearDev(p2, y)
-    d.apply_linear(regime)
+    _apply(d, regime)
     assert np.array_equal(host_bits(d.y), clean)
 
 
@@ -164,10 +200,10 @@ def test_position_permutation_and_rerun_bit_exact(regime):
     p = W.random_linear(12, 120, 256, (32,), 3, 16, ranks=[16, 8, 16])
     _skip_unsupported(p, regime)
     d = LinearDev(p)
-    d.apply_linear(regime)
+    _apply(d, regime)
     first = host_bits(d.y)
     d2 = LinearDev(p)
-    d2.apply_linear(regime)
+    _apply(d2, regime)
     assert np.array_equal(host_bits(d2.y), first)
     rng = np.random.default_rng(3)
     to = p.token_order.copy()
@@ -175,7 +211,7 @@ def test_position_permutation_and_rerun_bit_exact(regime):
         lo, hi = p.slot_indptr[s], p.slot_indptr[s + 1]
         to[lo:hi] = rng.permutation(to[lo:hi])
     d3 = LinearDev(W.LinearProblem(**{**p.__dict__, "token_order": to}))
-    d3.apply_linear(regime)
+    _apply(d3, regime)
     assert np.array_equal(host_bits(d3.y), first)
 
 
@@ -187,7 +223,7 @@ def test_shrink_and_expand(regime):
     d = LinearDev(p)
     SR = p.num_slices * p.R
     h = t.full((p.T, SR), float("nan"), dtype=t.float32, device="cuda")
-    d.shrink(h, regime)
+    d.shrink(h, min(int(regime), L.LORA_REGIME_SGMV))
     h_dev = h.cpu().numpy().astype(np.float64)
     h_ref, mask, flags = O.shrink(_f64(p.x), _f64(p.a), p.token_order, p.slot_indptr, p.ranks,
                                   p.R, p.num_slices)
@@ -199,7 +235,7 @@ def test_shrink_and_expand(regime):
     # expand from an fp32 h
     h32 = np.where(mask, h_ref, 0.0).astype(np.float32)
     h_in = t.from_numpy(h32).cuda()
-    d.expand(h_in, regime)
+    d.expand(h_in, min(int(regime), L.LORA_REGIME_SGMV))
     y_ref, touched, f2 = O.expand(_f64(p.y), h32.astype(np.float64), _f64(p.b), p.token_order,
                                   p.slot_indptr, p.ranks, p.scalings, p.out_slices, p.R)
     out = host_bits(d.y)
@@ -233,7 +269,7 @@ def test_apply_embedding(regime, seed):
                         bad_id_frac=0.1, dead_frac=0.05)
     _skip_unsupported(p, regime, shrink=False)
     d = LinearDev(p)
-    d.apply_embedding(regime)
+    d.apply_embedding(min(int(regime), L.LORA_REGIME_SGMV))
     y_ref, touched, flags = O.apply_embedding(p.ids, _f64(p.y), _f64(p.a), _f64(p.b),
                                               p.token_order, p.slot_indptr, p.ranks, p.scalings,
                                               p.out_slices, p.R, p.n_in)
@@ -243,7 +279,7 @@ def test_apply_embedding(regime, seed):
     assert_rows_bit_identical(out, p.y, ~touched, "embedding untouched")
     zero = np.zeros_like(p.y)
     d0 = LinearDev(p, zero)
-    d0.apply_embedding(regime)
+    d0.apply_embedding(min(int(regime), L.LORA_REGIME_SGMV))
     y0, _, _ = O.apply_embedding(p.ids, _f64(zero), _f64(p.a), _f64(p.b), p.token_order,
                                  p.slot_indptr, p.ranks, p.scalings, p.out_slices, p.R, p.n_in)
     assert_close(_f64(host_bits(d0.y)), y0, "embedding y=0")
@@ -315,7 +351,7 @@ def test_bad_addressing_flags(regime):
                            "ranks": ranks})
     _skip_unsupported(q, regime)
     d = LinearDev(q)
-    d.apply_linear(regime)
+    _apply(d, regime)
     y_ref, touched, flags = O.apply_linear(_f64(q.x), _f64(q.y), _f64(q.a), _f64(q.b), to,
                                            indptr, ranks, q.scalings, q.out_slices, q.R)
     out = host_bits(d.y)
@@ -380,31 +416,27 @@ def test_workload_decode_qkv_full():
     _check_linear(p, L.LORA_REGIME_AUTO, y_bits=np.zeros_like(p.y), what="decode y=0")
 
 
-def _sampled_oracle(p, tokens, y_bits):
-    """The oracle on a subset of tokens: the same addressing restricted to them."""
-    keep = np.zeros(p.T, dtype=bool)
-    keep[tokens] = True
-    slot_of = np.where(keep, p.slot_of, -1)
-    to, ip = W.csr_by_slot(slot_of, p.slots)
-    return O.apply_linear(_f64(p.x), _f64(y_bits), _f64(p.a), _f64(p.b), to, ip, p.ranks,
-                          p.scalings, p.out_slices, p.R)
+def _oracle_rows(p, tokens, y_bits):
+    """The oracle on a subset of tokens, as a problem of its own: their x and y
+    rows, their slots, the same adapters.  Returns y_ref for those rows."""
+    tokens = np.asarray(tokens)
+    to, ip = W.csr_by_slot(p.slot_of[tokens], p.slots)
+    y_ref, _, _ = O.apply_linear(_f64(p.x[tokens]), _f64(y_bits[tokens]), _f64(p.a), _f64(p.b),
+                                 to, ip, p.ranks, p.scalings, p.out_slices, p.R)
+    return y_ref
 
 
-def test_workload_prefill_gate_up_sampled():
+def test_workload_prefill_gate_up_full():
+    """Every row of y at the full prefill size (8192 tokens, out 28672) against
+    the fp64 oracle, element by element, in chunks of 1024 tokens."""
     p = W.prefill_gate_up(0)
     d = LinearDev(p)
     d.apply_linear(L.LORA_REGIME_AUTO)
     out = host_bits(d.y)
-    rng = np.random.default_rng(0)
-    tokens = rng.choice(p.T, size=96, replace=False)
-    y_ref, touched, _ = _sampled_oracle(p, tokens, p.y)
     assert read_flags(d.flags) == 0
-    assert_close(_f64(out[tokens]), y_ref[tokens], "prefill sampled")
-    # rows of the first and last segment positions (tile edges)
-    edges = p.token_order[np.unique(np.concatenate([p.slot_indptr[:-1],
-                                                    np.maximum(p.slot_indptr[1:] - 1, 0)]))]
-    y_e, _, _ = _sampled_oracle(p, edges, p.y)
-    assert_close(_f64(out[edges]), y_e[edges], "prefill segment edges")
+    for c0 in range(0, p.T, 1024):
+        rows = np.arange(c0, min(p.T, c0 + 1024))
+        assert_close(_f64(out[rows]), _oracle_rows(p, rows, p.y), f"prefill rows {c0}..")
 
 
 def test_workload_embedding_full():
@@ -439,7 +471,7 @@ def test_workload_moe_full():
 def _chain_problems(regime):
     # Three fused calls on one y: each reads the y the previous call wrote,
     # with its own x, adapters and slot layout.
-    if regime == L.LORA_REGIME_SGMV:
+    if int(regime) == L.LORA_REGIME_SGMV:
         return [W.random_linear(910 + k, 1200, 256, (128, 64), 4, 32, ranks=[32, 16, 8, 32],
                                 dead_frac=0.05) for k in range(3)]
     return [W.random_linear(900 + k, 256, 512, (256, 128, 64), 12, 16, ranks=None,
@@ -464,7 +496,9 @@ def test_launch_overlap_dependent_chain(regime, graph):
     ps = _chain_problems(regime)
     devs = [LinearDev(p) for p in ps]
     ws_bytes = max(L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R,
-                                          p.num_slices, regime) for p in ps)
+                                          p.num_slices, int(regime)) for p in ps)
+    if not regime.workspace:
+        ws_bytes = 0
     ws = t.zeros(max(ws_bytes, 16) // 4, dtype=t.float32, device="cuda")
     y = devs[0].y
     y0 = host_bits(y).copy()
@@ -475,7 +509,7 @@ def test_launch_overlap_dependent_chain(regime, graph):
                 p = d.p
                 L.lora_apply_linear(d.x, y, d.a, d.b, d.ranks, d.scalings, d.token_order,
                                     d.slot_indptr, p.T, p.n_in, p.slots, p.R, p.out_slices,
-                                    regime=regime, workspace=ws if ws_bytes else None,
+                                    regime=int(regime), workspace=ws if ws_bytes else None,
                                     workspace_bytes=ws_bytes, err_flags=d.flags)
         if graph:
             run()                                   # warm the launch caches outside capture
@@ -495,3 +529,44 @@ def test_launch_overlap_dependent_chain(regime, graph):
     assert_close(_f64(host_bits(y)), _f64(ref), "chain")
     assert all(read_flags(d.flags) == 0 for d in devs)
 
+
+
+# ---------------------------------------------------------------------------
+# The split kernel's bounded wait
+# ---------------------------------------------------------------------------
+
+def test_split_wait_runs_out_and_is_flagged():
+    """The BGMV_SPLIT kernel's bounded wait, made to run out without any fault:
+    the host sets the first work item's counter
+    in the workspace so that it never equals that item's number of shrink
+    pieces.  With a 2 ms limit every expand piece of that item gives up,
+    LORA_FLAG_TIMEOUT is raised, those rows of y are left as they were, every
+    other row is right, the call returns, and the counters end zeroed: the same
+    workspace then gives the oracle's result."""
+    t = torch()
+    p = W.decode_qkv(3)
+    ws_bytes = L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R, p.num_slices,
+                                      L.LORA_REGIME_BGMV_SPLIT)
+    ws = t.zeros(ws_bytes // 4, dtype=t.int32, device="cuda")
+    ws[0] = 1 << 30                    # item 0's counter: out of reach
+    d = LinearDev(p)
+    prev = L.lora_set_wait_limit_ns(2_000_000)
+    try:
+        d.apply_linear(L.LORA_REGIME_BGMV_SPLIT, workspace=ws)
+        t.cuda.synchronize()
+    finally:
+        L.lora_set_wait_limit_ns(prev)
+    assert read_flags(d.flags) == L.LORA_FLAG_TIMEOUT
+    # item 0: the 32 smallest token ids of the first slot with tokens
+    s0 = next(s for s in range(p.slots) if p.slot_indptr[s + 1] > p.slot_indptr[s])
+    toks0 = np.sort(p.token_order[p.slot_indptr[s0]:p.slot_indptr[s0 + 1]])[:32]
+    out = host_bits(d.y)
+    assert_rows_bit_identical(out, p.y, toks0, "timed-out item")
+    y_ref, touched, _ = _oracle_linear(p)
+    rest = np.setdiff1d(np.nonzero(touched)[0], toks0)
+    assert_close(_f64(out[rest]), y_ref[rest], "other items")
+    assert int(ws[:1024].abs().sum().item()) == 0     # counters zeroed again
+    d2 = LinearDev(p)
+    d2.apply_linear(L.LORA_REGIME_BGMV_SPLIT, workspace=ws)
+    assert read_flags(d2.flags) == 0
+    assert_close(_f64(host_bits(d2.y)), y_ref, "rerun on the same workspace")
