@@ -36,6 +36,10 @@ What it computes, and where each rule comes from (page title, section):
   independent, so the result equals one fold.
 * same page, ``apply_expert_lora_sorted``: the expert fold adds each adapted
   expert's delta onto its contiguous row block of the sorted output, in place.
+* same page, ``apply_router_lora`` and its module text: the router (``mlp.gate``)
+  adapter's delta is one delta fold onto the ``[n, num_experts]`` routing
+  logits, in place, before top-k selection; ``spark_model/lora/target.rs``,
+  ``router_dims``: the router projection is ``[num_experts, hidden]``.
 
 Readings where the pages are silent (each one is listed with its reason in the
 design notes of the repository):
@@ -377,6 +381,32 @@ def expert_apply(x, y, a, b, pair_index, ranks, scalings, row_slot, expert_offse
                             pair_index, ranks, scalings, row_slot, slots,
                             num_experts, num_pairs, R, out_slices)
     return y_ref, touched, flags
+
+
+# ---------------------------------------------------------------------------
+# Router fold
+# ---------------------------------------------------------------------------
+
+def apply_router(router_in, logits, a, b, token_order, slot_indptr, ranks, scalings, R):
+    """The router adapter's delta onto the routing logits, before top-k
+    (``apply_router_lora``): ``logits [T, E] += s * (router_in @ A^T) @ B^T`` per
+    token's slot, with ``a [slots, R, hidden]`` and ``b [slots, E, R]``.  The
+    page folds it with the same delta routine as a dense projection, so it is
+    the fused apply with a single output slice of ``E`` columns.  Returns
+    ``(logits_ref, touched, flags)``."""
+    E = logits.shape[1]
+    return apply_linear(router_in, logits, a, b, token_order, slot_indptr, ranks, scalings,
+                        (E,), R)
+
+
+def top_k_experts(logits, k):
+    """The ``k`` experts with the largest logits per token, largest first (ties
+    to the lower expert id): the selection that follows the router fold."""
+    out = []
+    for row in np.asarray(logits, dtype=np.float64):
+        order = sorted(range(len(row)), key=lambda e: (-row[e], e))
+        out.append(order[:k])
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -104,6 +104,26 @@ def test_adapted_experts_hand_example():
     assert flags == g["expected_flags"]
 
 
+def test_router_hand_example():
+    g = _load("router_hand.json")
+    args = dict(router_in=np.array(g["router_in"], float), logits=np.array(g["logits"], float),
+                a=np.array(g["a"], float), b=np.array(g["b"], float),
+                token_order=g["token_order"], slot_indptr=g["slot_indptr"], ranks=g["ranks"],
+                scalings=g["scalings"], R=g["R"])
+    out, touched, flags = O.apply_router(**args)
+    assert flags == 0
+    assert np.array_equal(out, np.array(g["expected_logits"], float))
+    assert list(touched) == g["expected_touched"]
+    # the element-by-element definition agrees
+    brute, bflags = O.brute_apply_linear(args["router_in"], args["logits"], args["a"],
+                                         args["b"], g["token_order"], g["slot_indptr"],
+                                         g["ranks"], g["scalings"], (g["num_experts"],), g["R"])
+    assert bflags == 0 and np.array_equal(brute, out)
+    # the fold comes before top-k: it changes token 0's choice
+    assert O.top_k_experts(args["logits"], 2) == g["expected_top2_before"]
+    assert O.top_k_experts(out, 2) == g["expected_top2_after"]
+
+
 def test_expert_fold_hand_example():
     g = _load("expert_fold_hand.json")
     args = dict(x=np.array(g["x"], float), y=np.array(g["y"], float),
