@@ -255,14 +255,19 @@ lora_status lora_expand(void* y, const float* h, const void* b, const int32_t* r
   return ok();
 }
 
-lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
-                              const int32_t* ranks, const float* scalings,
+}  // extern "C"
+
+namespace {
+
+// The fused shrink + expand behind lora_apply_linear and lora_apply_router;
+// `op` names the entry point in error messages.
+lora_status apply_linear_impl(const char* op, const void* x, void* y, const void* a,
+                              const void* b, const int32_t* ranks, const float* scalings,
                               const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
                               int32_t in_features, int32_t slots, int32_t R,
                               const int32_t* out_slices, int32_t num_slices, int32_t regime,
                               void* workspace, size_t workspace_bytes, uint32_t* err_flags,
                               void* stream) {
-  const char* op = "lora_apply_linear";
   lora::BgmvParams p = {};
   int out = 0;
   lora_status st = check_common(op, T, in_features, slots, R, num_slices, out_slices, true,
@@ -339,6 +344,42 @@ lora_status lora_apply_linear(const void* x, void* y, const void* a, const void*
                                       linear_items_bound(T, slots, lora::kFusedTile), s, &why);
   if (err != cudaSuccess) return cuda_fail(err, op, why);
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+lora_status lora_apply_linear(const void* x, void* y, const void* a, const void* b,
+                              const int32_t* ranks, const float* scalings,
+                              const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
+                              int32_t in_features, int32_t slots, int32_t R,
+                              const int32_t* out_slices, int32_t num_slices, int32_t regime,
+                              void* workspace, size_t workspace_bytes, uint32_t* err_flags,
+                              void* stream) {
+  return apply_linear_impl("lora_apply_linear", x, y, a, b, ranks, scalings, token_order,
+                           slot_indptr, T, in_features, slots, R, out_slices, num_slices, regime,
+                           workspace, workspace_bytes, err_flags, stream);
+}
+
+lora_status lora_apply_router(const void* router_in, void* gate_logits, const void* a,
+                              const void* b, const int32_t* ranks, const float* scalings,
+                              const int32_t* token_order, const int32_t* slot_indptr, int32_t T,
+                              int32_t hidden, int32_t slots, int32_t R, int32_t num_experts,
+                              int32_t regime, void* workspace, size_t workspace_bytes,
+                              uint32_t* err_flags, void* stream) {
+  const char* op = "lora_apply_router";
+  if (hidden <= 0 || hidden % 8 != 0)
+    return fail(LORA_ERR_INVALID, "%s: hidden = %d must be a positive multiple of 8", op, hidden);
+  if (num_experts <= 0 || num_experts % 8 != 0)
+    return fail(LORA_ERR_INVALID, "%s: num_experts = %d must be a positive multiple of 8", op,
+                num_experts);
+  // one slice of num_experts logit columns: the routing logits are the output
+  // of the router projection
+  const int32_t out_slices[1] = {num_experts};
+  return apply_linear_impl(op, router_in, gate_logits, a, b, ranks, scalings,
+                           token_order, slot_indptr, T, hidden, slots, R, out_slices, 1, regime,
+                           workspace, workspace_bytes, err_flags, stream);
 }
 
 lora_status lora_gather_shrink(const int32_t* ids, float* h, const void* a, const int32_t* ranks,

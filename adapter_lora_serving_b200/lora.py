@@ -53,6 +53,8 @@ _SIGS = [
      [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _Z, _P, _P]),
     ("lora_apply_linear_noalloc", _I,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _P]),
+    ("lora_apply_router", _I,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P]),
     ("lora_gather_shrink", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     ("lora_apply_embedding", _I,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _P]),
@@ -162,6 +164,16 @@ def lora_apply_linear_noalloc(x, y, a, b, ranks, scalings, token_order, slot_ind
                                             _ptr(slot_indptr), T, in_features, slots, R,
                                             _slices(out_slices), len(out_slices), regime,
                                             _ptr(err_flags), _stream(stream)))
+
+
+def lora_apply_router(router_in, gate_logits, a, b, ranks, scalings, token_order, slot_indptr,
+                      T, hidden, slots, R, num_experts, regime=LORA_REGIME_AUTO, workspace=None,
+                      workspace_bytes=0, err_flags=None, stream=None):
+    _check(load().lora_apply_router(_ptr(router_in), _ptr(gate_logits), _ptr(a), _ptr(b),
+                                    _ptr(ranks), _ptr(scalings), _ptr(token_order),
+                                    _ptr(slot_indptr), T, hidden, slots, R, num_experts, regime,
+                                    _ptr(workspace), workspace_bytes, _ptr(err_flags),
+                                    _stream(stream)))
 
 
 def lora_gather_shrink(ids, h, a, ranks, token_order, slot_indptr, T, vocab, slots, R,

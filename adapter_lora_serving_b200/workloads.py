@@ -355,6 +355,30 @@ def moe_expert(seed=0, T=2048, num_experts=128, top_k=8, hidden=2048, inter=768,
     return gu, dn
 
 
+def moe_router(seed=0, T=2048, num_experts=128, hidden=2048, slots=4, requests=16, R=16,
+               scaling=2.0):
+    """Router LoRA on the MoE layer above: the routing logits [T=2048, 128 experts]
+    of hidden 2048 take each token's router (mlp.gate) adapter delta before
+    top-k.  16 requests of 128 tokens, each with a slot uniform in 4 slots;
+    R = 16, rank per slot uniform in {8, 16}, scaling 2; router input and
+    logits ~ N(0,1), A,B ~ N(0,0.02).  One output slice of 128 columns."""
+    rng = np.random.default_rng(6000 + seed)
+    per_req = T // requests
+    req_slot = rng.integers(0, slots, size=requests)
+    slot_of = np.repeat(req_slot, per_req)
+    if len(slot_of) < T:
+        slot_of = np.concatenate([slot_of, np.full(T - len(slot_of), req_slot[-1])])
+    token_order, slot_indptr = csr_by_slot(slot_of, slots)
+    ranks = rng.choice([8, 16], size=slots).astype(np.int32)
+    scalings = np.full(slots, scaling, dtype=np.float32)
+    x = _normal_bf16(rng, (T, hidden), 1.0)
+    a = _normal_bf16(rng, (slots, R, hidden), 0.02)
+    b = _normal_bf16(rng, (slots, num_experts, R), 0.02)
+    y = _normal_bf16(rng, (T, num_experts), 1.0)
+    return LinearProblem("moe_router", T, hidden, (num_experts,), slots, R, x, a, b, y, ranks,
+                         scalings, token_order, slot_indptr, slot_of)
+
+
 def random_moe(seed, rows_per_expert_max, num_experts, n_in, out_slices, slots, R,
                ranks=None, adapted_frac=0.5, no_slot_frac=0.1):
     """A small MoE fold problem with ragged expert row blocks (tests)."""
@@ -393,4 +417,5 @@ WORKLOADS = {
     "prefill_gate_up": prefill_gate_up,
     "embedding": embedding,
     "moe_expert": moe_expert,
+    "moe_router": moe_router,
 }

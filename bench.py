@@ -45,6 +45,8 @@ DESCR = {
                  "slots=8, R=16, ranks {8,16}",
     "moe_expert": "MoE expert LoRA: 128 experts, hidden=2048, moe_inter=768, top-8 of T=2048 "
                   "-> 16384 sorted rows, 4 slots, 25% experts adapted, R=16; gate/up + down folds",
+    "moe_router": "MoE router LoRA: routing logits [T=2048, 128 experts], hidden=2048, "
+                  "4 slots, R=16, ranks {8,16}; fold before top-k",
 }
 
 
@@ -210,6 +212,12 @@ class Workload:
                                    d["token_order"], d["slot_indptr"], p.T, p.n_in, p.slots, p.R,
                                    p.out_slices, stream=stream)
             return
+        if self.name == "moe_router":
+            L.lora_apply_router(d["x"], d["y"], d["a"], d["b"], d["ranks"], d["scalings"],
+                                d["token_order"], d["slot_indptr"], p.T, p.n_in, p.slots, p.R,
+                                p.out, workspace=d["ws"], workspace_bytes=d["ws_bytes"],
+                                stream=stream)
+            return
         L.lora_apply_linear(d["x"], d["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                             d["token_order"], d["slot_indptr"], p.T, p.n_in, p.slots, p.R,
                             p.out_slices, workspace=d["ws"], workspace_bytes=d["ws_bytes"],
@@ -219,7 +227,7 @@ class Workload:
 def n_sets_for(name):
     """Input sets so that one rotation is larger than twice the L2."""
     per = {"tiny_linear": 0.13e6, "decode_qkv": 21.6e6, "prefill_gate_up": 1.2e9,
-           "embedding": 70e6, "moe_expert": 110e6}[name]
+           "embedding": 70e6, "moe_expert": 110e6, "moe_router": 9.2e6}[name]
     return max(1, min(64, int(math.ceil(2.2 * L2_BYTES / per))))
 
 
@@ -414,6 +422,10 @@ def time_e2e(torch, wl, steps):
             L.lora_apply_embedding(dev["ids"], dev["y"], d["a"], d["b"], d["ranks"],
                                    d["scalings"], dev["token_order"], dev["slot_indptr"], p.T,
                                    p.n_in, p.slots, p.R, p.out_slices)
+        elif wl.name == "moe_router":
+            L.lora_apply_router(dev["x"], dev["y"], d["a"], d["b"], d["ranks"], d["scalings"],
+                                dev["token_order"], dev["slot_indptr"], p.T, p.n_in, p.slots,
+                                p.R, p.out, workspace=d["ws"], workspace_bytes=d["ws_bytes"])
         else:
             L.lora_apply_linear(dev["x"], dev["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                                 dev["token_order"], dev["slot_indptr"], p.T, p.n_in, p.slots,
@@ -484,6 +496,8 @@ def oracle_step_fn(name, prob, frac=1.0, rng=None):
         if name == "embedding":
             O.apply_embedding(prob.ids, y, a, b, to, ip, prob.ranks, prob.scalings,
                               prob.out_slices, prob.R, prob.n_in)
+        elif name == "moe_router":
+            O.apply_router(x, y, a, b, to, ip, prob.ranks, prob.scalings, prob.R)
         else:
             O.apply_linear(x, y, a, b, to, ip, prob.ranks, prob.scalings, prob.out_slices,
                            prob.R)
@@ -533,7 +547,7 @@ def time_oracle(name, prob, budget_s=12.0, min_s=10.0):
 # Sources each kernel is built from: stored DRAM counters stay valid while
 # these files are unchanged.
 KERNEL_SOURCES = {
-    "bgmv_kernel": ["bgmv.cu", "common.cuh", "kernels.h"],
+    "bgmv_kernel": ["bgmv.cu", "common.cuh", "kernels.h", "expand_tile.cuh"],
     "sgmv_expand_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
     "sgmv_shrink_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
 }

@@ -162,6 +162,30 @@ LORA_API lora_status lora_apply_linear(const void* x, void* y, const void* a, co
                               void* stream);
 
 /*
+ * lora_apply_router -- the router LoRA fold (spark_model/lora/expert_apply.rs,
+ * apply_router_lora and its module text; router shape from
+ * spark_model/lora/target.rs, router_dims and the Router target): a MoE
+ * layer's routing logits take the delta of the router (mlp.gate) adapter of
+ * each token's slot, BEFORE top-k expert selection, so the selection sees
+ *   gate_logits[t, e] += scalings[slot] * sum_{r<rank} (router_in[t] @ a[slot, r]^T) * b[slot, e, r].
+ * router_in [T, hidden] bf16 (the router's input); gate_logits [T, num_experts]
+ * bf16, updated in place; a [slots, R, hidden] bf16; b [slots, num_experts, R]
+ * bf16; addressing, ranks and scalings as for lora_apply_linear.  It is
+ * lora_apply_linear with in_features = hidden and one output slice of
+ * num_experts columns, run by the same kernels (regime, workspace and flags
+ * behave the same: size the workspace with lora_workspace_bytes(
+ * LORA_OP_APPLY_LINEAR, T, slots, R, 1, regime)).  hidden and num_experts must
+ * be positive multiples of 8 (LORA_ERR_INVALID otherwise).
+ */
+LORA_API lora_status lora_apply_router(const void* router_in, void* gate_logits, const void* a,
+                                       const void* b, const int32_t* ranks,
+                                       const float* scalings, const int32_t* token_order,
+                                       const int32_t* slot_indptr, int32_t T, int32_t hidden,
+                                       int32_t slots, int32_t R, int32_t num_experts,
+                                       int32_t regime, void* workspace, size_t workspace_bytes,
+                                       uint32_t* err_flags, void* stream);
+
+/*
  * lora_gather_shrink -- LoraBackend.gather_shrink:
  *   h[t, i*R + r] = a[slot(t), i*R + r, ids[t]]  (r < rank)
  * ids [T] int32 token ids; a [slots, num_slices*R, vocab] bf16; h [T, num_slices*R]

@@ -77,6 +77,20 @@ class LinearDev:
                             out_slices or p.out_slices, regime=regime, workspace=workspace,
                             workspace_bytes=ws_bytes, err_flags=self.flags)
 
+    def apply_router(self, regime=L.LORA_REGIME_AUTO):
+        """lora_apply_router on a one-slice problem (y = the routing logits)."""
+        p = self.p
+        assert p.num_slices == 1
+        ws_bytes = L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R, 1, regime)
+        workspace = None
+        if ws_bytes:
+            t = torch()
+            workspace = t.zeros(ws_bytes // 4 + 4, dtype=t.float32, device="cuda")
+        L.lora_apply_router(self.x, self.y, self.a, self.b, self.ranks, self.scalings,
+                            self.token_order, self.slot_indptr, p.T, p.n_in, p.slots, p.R,
+                            p.out, regime=regime, workspace=workspace, workspace_bytes=ws_bytes,
+                            err_flags=self.flags)
+
     def shrink(self, h, regime=L.LORA_REGIME_AUTO):
         p = self.p
         L.lora_shrink(self.x, h, self.a, self.ranks, self.token_order, self.slot_indptr, p.T,

@@ -104,6 +104,25 @@ def test_other_entry_points_validate(lib):
                                 None) == L.LORA_ERR_INVALID
 
 
+def test_router_validates(lib):
+    # router_in, gate_logits, a, b, ranks, scalings, token_order, slot_indptr,
+    # T, hidden, slots, R, num_experts, regime, workspace, bytes, flags, stream
+    def router(**kw):
+        args = dict(T=16, hidden=64, slots=2, R=16, num_experts=64)
+        args.update(kw)
+        return lib.lora_apply_router(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, args["T"],
+                                     args["hidden"], args["slots"], args["R"],
+                                     args["num_experts"], L.LORA_REGIME_BGMV, None, 0, None,
+                                     None)
+    assert router(num_experts=60) == L.LORA_ERR_INVALID
+    assert "num_experts" in lib.lora_last_error().decode()
+    assert router(num_experts=0) == L.LORA_ERR_INVALID
+    assert router(hidden=100) == L.LORA_ERR_INVALID
+    assert lib.lora_last_error().decode().startswith("lora_apply_router")
+    assert router(R=12) == L.LORA_ERR_INVALID
+    assert router(T=0) == L.LORA_OK
+
+
 def test_status_strings(lib):
     for code, name in [(0, "LORA_OK"), (1, "LORA_ERR_INVALID"), (2, "LORA_ERR_UNSUPPORTED"),
                        (3, "LORA_ERR_WORKSPACE"), (4, "LORA_ERR_CUDA")]:
