@@ -93,6 +93,10 @@ int resolve(int regime, int op, int T, int slots, int R, int S, int in_features 
   if (regime == LORA_REGIME_BGMV || regime == LORA_REGIME_SGMV) return regime;
   if (regime == LORA_REGIME_BGMV_SPLIT)
     return op == LORA_OP_APPLY_LINEAR ? LORA_REGIME_BGMV_SPLIT : LORA_REGIME_BGMV;
+  if (regime == LORA_REGIME_STREAM)
+    return op == LORA_OP_APPLY_EMBEDDING ? LORA_REGIME_STREAM : LORA_REGIME_BGMV;
+  // the embedding: stream the output rows through shared memory
+  if (op == LORA_OP_APPLY_EMBEDDING && lora::stream_supported(R)) return LORA_REGIME_STREAM;
   const bool needs_shrink = (op == LORA_OP_SHRINK || op == LORA_OP_APPLY_LINEAR);
   // Many tokens per slot on average: tensor-core tiles over slot segments.
   if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024 &&
@@ -155,6 +159,7 @@ int32_t lora_resolve_regime(int32_t op, int32_t T, int32_t slots, int32_t R, int
 
 int32_t lora_plan_tile(int32_t op, int32_t regime) {
   if (op == LORA_OP_EXPERT_APPLY) return lora::kTT;
+  if (op == LORA_OP_APPLY_EMBEDDING && regime == LORA_REGIME_STREAM) return lora::kStRows;
   if (regime == LORA_REGIME_SGMV) return lora::kSgmvTileM;
   if (op == LORA_OP_APPLY_LINEAR) return lora::kFusedTile;
   return lora::kTT;
@@ -435,6 +440,20 @@ lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, con
     return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
   const int reg = resolve(regime, LORA_OP_APPLY_EMBEDDING, T, slots, R, num_slices);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (reg == LORA_REGIME_STREAM) {
+    if (!lora::stream_supported(R))
+      return fail(LORA_ERR_UNSUPPORTED, "%s: the STREAM regime needs roundup(R, 16) <= %d", op,
+                  lora::kStMaxRp);
+    lora::StreamParams q = {};
+    q.ids = ids; q.y = y; q.a = a; q.b = b; q.ranks = ranks; q.scalings = scalings;
+    q.token_order = token_order; q.slot_indptr = slot_indptr; q.flags = err_flags;
+    q.T = T; q.vocab = vocab; q.slots = slots; q.R = R; q.S = num_slices; q.out = out;
+    for (int i = 0; i <= LORA_MAX_SLICES; ++i) q.slice_off[i] = p.slice_off[i];
+    const char* why = nullptr;
+    cudaError_t err = lora::stream_embed_launch(q, s, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
       return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);

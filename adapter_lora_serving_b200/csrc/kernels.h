@@ -286,6 +286,54 @@ inline size_t split_workspace_bytes(int T, int slots, int R, int S) {
 
 cudaError_t split_launch(const SplitParams& p, cudaStream_t stream, const char** why);
 
+// ---------------------------------------------------------------------------
+// Streamed embedding apply (stream.cu).  The output columns are cut into
+// blocks of at most W columns (one slice each) and the token positions into
+// equal shares; CTA c (one per SM) takes block run c % bsplit and position
+// share c / bsplit, cuts the live slots' segments inside its share into
+// groups of kStRows positions and walks its (block, group) units block by
+// block.  A producer warp bulk-copies a B block into a ring of kStBBufs
+// buffers whenever the (slot, block) changes; consumer warps hold their B
+// fragments in registers, keep the y rows of the next kStDepth units in
+// flight in registers, apply the gathered h with warp MMAs and store y.
+// ---------------------------------------------------------------------------
+constexpr int kStRows = 16;       // positions per group (one MMA row tile)
+constexpr int kStConsumers = 16;  // consumer warps (one 32-column chunk each)
+constexpr int kStThreads = 32 * (1 + kStConsumers);
+constexpr int kStDepth = 4;       // units of y in flight per consumer warp
+constexpr int kStBBufs = 4;       // B blocks in flight
+constexpr int kStMaxRp = 64;      // roundup(R, 16) limit
+constexpr int kStMaxGroups = 64;  // groups per table window
+constexpr int kStSpec = 2048;     // token_order entries a CTA reads ahead at most
+
+struct StreamParams {
+  const int* ids;
+  void* y;
+  const void* a;
+  const void* b;
+  const int* ranks;
+  const float* scalings;
+  const int* token_order;
+  const int* slot_indptr;
+  uint32_t* flags;
+  uint64_t wait_ns;
+  int T, vocab, slots, R, S, out;
+  int slice_off[LORA_MAX_SLICES + 1];
+  int block_off[LORA_MAX_SLICES + 1];  // exclusive prefix of column blocks per slice
+  int nblocks;                         // column blocks of all slices
+  int W;                               // columns per block at most
+  int bsplit;                          // block runs (divides the grid)
+  int gtab;                            // groups per table window
+  int bbytes;                          // bytes of one B buffer (W * R * 2)
+  int off_prefix, off_scratch, off_spec, off_ctok, off_cval, off_gmeta, off_htab, off_bbuf;
+  int smem;
+};
+
+// The streamed embedding takes roundup(R, 16) <= kStMaxRp.
+inline bool stream_supported(int R) { return round_up_i(R, 16) <= kStMaxRp; }
+// Fills the layout fields of p (from T, slots, R, S and slice_off) and launches.
+cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char** why);
+
 // Workspace bytes lora_apply_linear needs for these shapes in `regime` (AUTO
 // resolved with the real in_features), 0 if none (api.cu).
 size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,

@@ -32,6 +32,7 @@ LORA_REGIME_AUTO = 0
 LORA_REGIME_BGMV = 1
 LORA_REGIME_SGMV = 2
 LORA_REGIME_BGMV_SPLIT = 3
+LORA_REGIME_STREAM = 4
 
 LORA_OP_SHRINK = 0
 LORA_OP_EXPAND = 1

@@ -550,6 +550,7 @@ KERNEL_SOURCES = {
     "bgmv_kernel": ["bgmv.cu", "common.cuh", "kernels.h", "expand_tile.cuh"],
     "sgmv_expand_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
     "sgmv_shrink_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
+    "stream_embed_kernel": ["stream.cu", "common.cuh", "kernels.h", "expand_tile.cuh"],
 }
 
 

@@ -89,6 +89,9 @@ typedef enum {
 #define LORA_REGIME_SGMV 2   /* many tokens per slot: tcgen05/TMEM tiles over slot segments */
 #define LORA_REGIME_BGMV_SPLIT 3  /* few tokens per slot, the work split by bytes over every SM
                                      (lora_apply_linear only; needs a zeroed workspace) */
+#define LORA_REGIME_STREAM 4 /* output rows streamed through shared memory by bulk copies, the
+                                delta from warp MMAs (lora_apply_embedding only; AUTO's choice
+                                there) */
 
 #define LORA_MAX_SLICES 8
 #define LORA_MAX_SLOTS 4096
@@ -202,6 +205,9 @@ LORA_API lora_status lora_gather_shrink(const int32_t* ids, float* h, const void
  * lora_apply_embedding -- LoraBackend.apply_ with embedding=True (gather, then
  * expand; fused, h kept on chip).  A token whose id is outside [0, vocab)
  * contributes nothing and its row of y stays bit-identical.
+ * Regimes: AUTO and STREAM run one launch over every SM that streams the y rows
+ * of every live token through shared memory (roundup(R, 16) <= 64, else
+ * AUTO takes one of the others); BGMV and SGMV run those regimes' kernels.
  */
 LORA_API lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, const void* b,
                                  const int32_t* ranks, const float* scalings,

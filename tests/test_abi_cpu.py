@@ -149,6 +149,14 @@ def test_host_queries(lib):
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 8192, 16, 64, 2,
                                   L.LORA_REGIME_SGMV) == 4096 + 4 * 8192 * 64 * 2 * 4
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == L.LORA_REGIME_BGMV
+    # the embedding streams its output rows under AUTO (R up to 64)
+    assert L.lora_resolve_regime(L.LORA_OP_APPLY_EMBEDDING, 4096, 8, 16, 1) == \
+        L.LORA_REGIME_STREAM
+    assert L.lora_resolve_regime(L.LORA_OP_APPLY_EMBEDDING, 64, 8, 64, 2) == \
+        L.LORA_REGIME_STREAM
+    assert L.lora_resolve_regime(L.LORA_OP_APPLY_EMBEDDING, 64, 8, 72, 1) != \
+        L.LORA_REGIME_STREAM
+    assert L.lora_plan_tile(L.LORA_OP_APPLY_EMBEDDING, L.LORA_REGIME_STREAM) == 16
 
 
 def test_wait_limit_setting_roundtrip(lib):
