@@ -116,6 +116,16 @@ size_t apply_linear_need(int reg, int T, int in_features, int slots, int R, int 
   return 0;
 }
 
+// Workspace of the grouped expert fold: token_order [rows_cap], the group
+// tables (seg_lo, seg_hi, g_rank, g_scal; kMoeMaxGroups each), then the SGMV
+// partial h buffers.  0 when the shapes are not the SGMV kernels'.
+size_t expert_group_need(int rows_cap, int R, int S) {
+  if (rows_cap <= 0 || !lora::sgmv_supported(S, R)) return 0;
+  const size_t tok = ((size_t)rows_cap * 4 + 255) / 256 * 256;
+  const size_t tables = (size_t)4 * lora::kMoeMaxGroups * 4;
+  return tok + tables + lora::sgmv_workspace_bytes(rows_cap, R, S);
+}
+
 int linear_items_bound(int T, int slots, int tile) {
   const long long b = (long long)slots + ((long long)T + tile - 1) / tile;
   return (int)(b > (1LL << 30) ? (1LL << 30) : b);
@@ -167,6 +177,11 @@ int32_t lora_plan_tile(int32_t op, int32_t regime) {
 
 size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R, int32_t num_slices,
                             int32_t regime) {
+  if (op == LORA_OP_EXPERT_APPLY) {
+    // the grouped (tensor-core) fold; BGMV asks for the per-chunk kernel
+    if (regime == LORA_REGIME_BGMV || T <= 0 || R <= 0 || num_slices <= 0) return 0;
+    return expert_group_need(T, R, num_slices);
+  }
   if (op != LORA_OP_APPLY_LINEAR || T <= 0 || R <= 0 || num_slices <= 0) return 0;
   const int reg = resolve(regime, op, T, slots, R, num_slices);
   // in_features and out are not known here: size for the largest the split
@@ -450,7 +465,7 @@ lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, con
     q.T = T; q.vocab = vocab; q.slots = slots; q.R = R; q.S = num_slices; q.out = out;
     for (int i = 0; i <= LORA_MAX_SLICES; ++i) q.slice_off[i] = p.slice_off[i];
     const char* why = nullptr;
-    cudaError_t err = lora::stream_embed_launch(q, s, &why);
+    cudaError_t err = lora::stream_launch(q, s, true, &why);
     if (err != cudaSuccess) return cuda_fail(err, op, why);
     return ok();
   }
@@ -485,8 +500,6 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
                               const int32_t* out_slices, int32_t num_slices, void* workspace,
                               size_t workspace_bytes, uint32_t* err_flags, void* stream) {
   const char* op = "lora_expert_apply";
-  (void)workspace;
-  (void)workspace_bytes;
   lora::BgmvParams p = {};
   int out = 0;
   if (num_experts < 0 || num_experts > LORA_MAX_EXPERTS)
@@ -503,6 +516,46 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
   if (st != LORA_OK) return st;
   if (err_flags != nullptr && !aligned4(err_flags))
     return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t gneed = expert_group_need(rows_cap, R, num_slices);
+  if (workspace != nullptr && gneed > 0 && workspace_bytes >= gneed &&
+      (long long)slots * num_experts <= lora::kMoeMaxGroups && in_features >= 64 &&
+      lora::stream_supported(R)) {
+    // grouped fold: rows sorted by (slot, expert), then the SGMV shrink and
+    // expand over the groups' segments
+    if (!aligned16(workspace))
+      return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
+    const int G = slots * num_experts;
+    char* w = static_cast<char*>(workspace);
+    int* tok = reinterpret_cast<int*>(w);
+    int* seg_lo = reinterpret_cast<int*>(w + ((size_t)rows_cap * 4 + 255) / 256 * 256);
+    int* seg_hi = seg_lo + lora::kMoeMaxGroups;
+    int* g_rank = seg_hi + lora::kMoeMaxGroups;
+    float* g_scal = reinterpret_cast<float*>(g_rank + lora::kMoeMaxGroups);
+    float* hws = g_scal + lora::kMoeMaxGroups;
+    cudaError_t err = lora::moe_group_launch(expert_offsets, pair_index, row_slot, ranks,
+                                             scalings, rows_cap, num_experts, slots, num_pairs,
+                                             R, tok, seg_lo, seg_hi, g_rank, g_scal, err_flags, s);
+    if (err != cudaSuccess) return cuda_fail(err, op, nullptr);
+    const lora::SgmvGroups groups = {seg_hi, pair_index, num_pairs};
+    const char* why = nullptr;
+    // live groups are about the pairs in use: split the shrink to fill the SMs
+    const int ks = lora::sgmv_shrink_splits(0, num_pairs < G ? num_pairs : G, in_features);
+    err = lora::sgmv_shrink_launch(x_sorted, a, hws, g_rank, tok, seg_lo, rows_cap, in_features,
+                                   G, R, num_slices, err_flags, s, &why, ks, g_scal, &groups);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    // the expand: the groups are short (a few dozen rows), so their y rows are
+    // streamed with 16-row MMA tiles rather than tiled by 128
+    lora::StreamParams q = {};
+    q.h = hws; q.h_split = (size_t)rows_cap * num_slices * R; q.ksplit = ks;
+    q.y = y_sorted; q.b = b; q.ranks = g_rank; q.scalings = g_scal; q.token_order = tok;
+    q.slot_indptr = seg_lo; q.seg_hi = seg_hi; q.slot_map = pair_index; q.flags = err_flags;
+    q.T = rows_cap; q.vocab = 0; q.slots = G; q.R = R; q.S = num_slices; q.out = out;
+    for (int i = 0; i <= LORA_MAX_SLICES; ++i) q.slice_off[i] = p.slice_off[i];
+    err = lora::stream_launch(q, s, false, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
   if (!bgmv_fits(num_slices, R))
     return fail(LORA_ERR_UNSUPPORTED, "%s: num_slices*roundup(R,16) = %d > %d", op,
                 num_slices * lora::round_up_i(R, 16), lora::kMaxSRp);
@@ -510,7 +563,6 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
   p.scalings = scalings; p.row_slot = row_slot; p.expert_offsets = expert_offsets;
   p.flags = err_flags; p.T = rows_cap; p.in = in_features; p.slots = slots; p.R = R;
   p.S = num_slices; p.out = out; p.num_experts = num_experts; p.num_pairs = num_pairs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const char* why = nullptr;
   // one CTA per work item (a chunk of one expert's rows)
   const int bound = linear_items_bound(rows_cap, num_experts, lora::kTT);

@@ -265,11 +265,15 @@ LORA_DEV int block_inclusive_scan(int v, int* scratch, int* total) {
 // (scalings != nullptr), its scaling is nonzero.  Its positions are cut into
 // consecutive tiles of `tile`.  Writes prefix[0..slots] (exclusive prefix of
 // tile counts) to shared memory and returns the item count.  Flags for bad
-// segments and ranks are raised when `report` is set.
+// segments and ranks are raised when `report` is set.  The segment of slot s
+// is [slot_indptr[s], slot_indptr[s+1]), or [slot_indptr[s], seg_hi[s]) when
+// seg_hi is given (segments that need not abut, e.g. the MoE fold's
+// (slot, expert) groups).
 template <int NT>
 LORA_DEV int plan_linear(const int* __restrict__ slot_indptr, const int* __restrict__ ranks,
                          const float* __restrict__ scalings, int slots, int T, int R, int tile,
-                         int* prefix, int* scratch, uint32_t* flags, bool report) {
+                         int* prefix, int* scratch, uint32_t* flags, bool report,
+                         const int* __restrict__ seg_hi = nullptr) {
   uint32_t bad = 0;
   int carry = 0;
   if (threadIdx.x == 0) prefix[0] = 0;
@@ -278,7 +282,7 @@ LORA_DEV int plan_linear(const int* __restrict__ slot_indptr, const int* __restr
     int cnt = 0;
     if (s < slots) {
       const int lo = slot_indptr[s];
-      const int hi = slot_indptr[s + 1];
+      const int hi = seg_hi != nullptr ? seg_hi[s] : slot_indptr[s + 1];
       const int r = ranks[s];
       const bool seg_ok = lo >= 0 && lo <= hi && hi <= T;
       const bool rank_ok = r >= 0 && r <= R;

@@ -287,15 +287,16 @@ inline size_t split_workspace_bytes(int T, int slots, int R, int S) {
 cudaError_t split_launch(const SplitParams& p, cudaStream_t stream, const char** why);
 
 // ---------------------------------------------------------------------------
-// Streamed embedding apply (stream.cu).  The output columns are cut into
-// blocks of at most W columns (one slice each) and the token positions into
-// equal shares; CTA c (one per SM) takes block run c % bsplit and position
-// share c / bsplit, cuts the live slots' segments inside its share into
-// groups of kStRows positions and walks its (block, group) units block by
-// block.  A producer warp bulk-copies a B block into a ring of kStBBufs
-// buffers whenever the (slot, block) changes; consumer warps hold their B
-// fragments in registers, keep the y rows of the next kStDepth units in
-// flight in registers, apply the gathered h with warp MMAs and store y.
+// Streamed expand (stream.cu): the embedding target (h gathered from A by token
+// id) and the expand of a computed h (fp32 partial buffers, e.g. the grouped
+// MoE fold).  The positions of every slot that takes part are cut into row
+// groups of kStRows and the output columns into blocks of at most W columns
+// (one slice each); the (row group, block) units, row group by row group, are
+// split into equal runs, one per CTA (one per SM).  A producer warp
+// bulk-copies a B block into a ring of kStBBufs buffers whenever the (slot,
+// block) changes; consumer warps hold their B fragments in registers, keep
+// the y rows of the next kStDepth units in flight in registers, apply h with
+// warp MMAs and store y.
 // ---------------------------------------------------------------------------
 constexpr int kStRows = 16;       // positions per group (one MMA row tile)
 constexpr int kStConsumers = 16;  // consumer warps (one 32-column chunk each)
@@ -307,7 +308,10 @@ constexpr int kStMaxGroups = 64;  // groups per table window
 constexpr int kStSpec = 2048;     // token_order entries a CTA reads ahead at most
 
 struct StreamParams {
-  const int* ids;
+  const int* ids;             // embedding: token ids (h gathered from a)
+  const float* h;             // or: h partial buffers [ksplit][T][S*R] (fp32)
+  size_t h_split;             // elements between the partial buffers
+  int ksplit;
   void* y;
   const void* a;
   const void* b;
@@ -315,6 +319,8 @@ struct StreamParams {
   const float* scalings;
   const int* token_order;
   const int* slot_indptr;
+  const int* seg_hi;          // grouped addressing: segment ends, or nullptr
+  const int* slot_map;        // grouped addressing: b pair of each group, or nullptr
   uint32_t* flags;
   uint64_t wait_ns;
   int T, vocab, slots, R, S, out;
@@ -322,17 +328,29 @@ struct StreamParams {
   int block_off[LORA_MAX_SLICES + 1];  // exclusive prefix of column blocks per slice
   int nblocks;                         // column blocks of all slices
   int W;                               // columns per block at most
-  int bsplit;                          // block runs (divides the grid)
   int gtab;                            // groups per table window
   int bbytes;                          // bytes of one B buffer (W * R * 2)
-  int off_prefix, off_scratch, off_spec, off_ctok, off_cval, off_gmeta, off_htab, off_bbuf;
+  int off_prefix, off_scratch, off_spec, off_ctok, off_cval, off_gmeta, off_htab;
+  int off_bbuf;
   int smem;
 };
 
-// The streamed embedding takes roundup(R, 16) <= kStMaxRp.
+// The streamed kernels take roundup(R, 16) <= kStMaxRp.
 inline bool stream_supported(int R) { return round_up_i(R, 16) <= kStMaxRp; }
-// Fills the layout fields of p (from T, slots, R, S and slice_off) and launches.
-cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char** why);
+// Fills the layout fields of p (from T, slots, R, S and slice_off) and launches
+// (the programmatic edge to the preceding kernel only when allow_overlap).
+cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overlap,
+                          const char** why);
+
+// The MoE fold grouped by (slot, expert) (moe_group.cu): per adapted expert,
+// its rows sorted by slot into token_order, group g = s * num_experts + e owning
+// [seg_lo[g], seg_hi[g]) with rank g_rank[g] and scaling g_scal[g].
+constexpr int kMoeMaxGroups = 4096;   // slots * num_experts of the grouped fold
+cudaError_t moe_group_launch(const int* expert_offsets, const int* pair_index, const int* row_slot,
+                             const int* ranks, const float* scalings, int rows_cap,
+                             int num_experts, int slots, int num_pairs, int R, int* token_order,
+                             int* seg_lo, int* seg_hi, int* g_rank, float* g_scal,
+                             uint32_t* flags, cudaStream_t stream);
 
 // Workspace bytes lora_apply_linear needs for these shapes in `regime` (AUTO
 // resolved with the real in_features), 0 if none (api.cu).

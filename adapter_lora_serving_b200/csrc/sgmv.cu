@@ -55,6 +55,8 @@ struct ExpandParams {
   const float* scalings;
   const int* token_order;
   const int* slot_indptr;
+  const int* seg_hi;         // grouped addressing: segment ends, or nullptr
+  const int* slot_map;       // grouped addressing: a/b pair of each group, or nullptr
   uint32_t* flags;
   int T, vocab, slots, R, S, out;
   int span;                  // bytes per K-major row: 2*R (32, 64 or 128)
@@ -73,6 +75,8 @@ struct ShrinkParams {
   const float* scalings;     // nullptr: unscaled plan
   const int* token_order;
   const int* slot_indptr;
+  const int* seg_hi;         // grouped addressing: segment ends, or nullptr
+  const int* slot_map;       // grouped addressing: a/b pair of each group, or nullptr
   uint32_t* flags;
   int T, in, slots, R, S;
 };
@@ -104,6 +108,12 @@ LORA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag
 
 LORA_DEV uint32_t align1024(uint32_t v) { return (v + 1023u) & ~1023u; }
 
+// End of slot (or group) s's segment, and the a/b pair it uses.
+LORA_DEV int seg_end(const int* indptr, const int* seg_hi, int s) {
+  return seg_hi != nullptr ? seg_hi[s] : indptr[s + 1];
+}
+LORA_DEV int ab_of(const int* slot_map, int s) { return slot_map != nullptr ? slot_map[s] : s; }
+
 // Walks consecutive expand units without divisions: the item (and its slot
 // segment) is decoded only when the column chunks of an item run out.
 struct UnitCursor {
@@ -113,7 +123,7 @@ struct UnitCursor {
     item = it;
     s = find_segment(prefix, p.slots, it);
     p0 = p.slot_indptr[s] + (it - prefix[s]) * kTM;
-    n = max(0, min(kTM, p.slot_indptr[s + 1] - p0));
+    n = max(0, min(kTM, seg_end(p.slot_indptr, p.seg_hi, s) - p0));
   }
   LORA_DEV void set_chunk(const ExpandParams& p) {
     while (slice + 1 < p.S && p.chunk_off[slice + 1] <= cj) ++slice;
@@ -194,7 +204,7 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
   }
   const int items = plan_linear<kExThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
                                             p.R, kTM, prefix, scratch, p.flags,
-                                            blockIdx.x == 0);
+                                            blockIdx.x == 0, p.seg_hi);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -217,7 +227,8 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
             !wait_or_abort(&bempty[st], (uint32_t)((k / kNB - 1) & 1), abort_flag, p.flags))
           break;
         mbar_arrive_expect_tx(&bfull[st], tile_b);
-        tma_load_2d(bring + st * tile_b, &tmap_b, 0, U.s * p.out + U.col0, &bfull[st]);
+        tma_load_2d(bring + st * tile_b, &tmap_b, 0, ab_of(p.slot_map, U.s) * p.out + U.col0,
+                    &bfull[st]);
       }
     }
   } else if (warp == 1) {
@@ -363,7 +374,8 @@ sgmv_expand_kernel(const __grid_constant__ CUtensorMap tmap_b, const ExpandParam
                 for (int ks = 0; ks < p.ksplit; ++ks) val += hp[(size_t)ks * p.h_split];
               } else {
                 const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(p.a);
-                val = __bfloat162float(ab[((size_t)U.s * p.S * p.R + i * p.R + r) * p.vocab + id]);
+                val = __bfloat162float(
+                    ab[((size_t)ab_of(p.slot_map, U.s) * p.S * p.R + i * p.R + r) * p.vocab + id]);
               }
             }
             v[q] = val;
@@ -499,7 +511,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
   }
   const int items = plan_linear<kSgThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
                                             p.R, kTM, prefix, scratch, p.flags,
-                                            blockIdx.x == 0);
+                                            blockIdx.x == 0, p.seg_hi);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -516,7 +528,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
     ks = (int)(u - (long long)item * p.ksplit);
     s = find_segment(prefix, p.slots, item);
     p0 = p.slot_indptr[s] + (item - prefix[s]) * kTM;
-    n = max(0, min(kTM, p.slot_indptr[s + 1] - p0));
+    n = max(0, min(kTM, seg_end(p.slot_indptr, p.seg_hi, s) - p0));
     kb0 = min(nkb_total, ks * p.kb_per_split);
     kb1 = min(nkb_total, kb0 + p.kb_per_split);
   };
@@ -568,7 +580,7 @@ sgmv_shrink_kernel(const __grid_constant__ CUtensorMap tmap_a, const ShrinkParam
           for (int i = 0; i < p.S; ++i)
             for (int q = 0; q < groups; ++q)
               tma_load_2d(at + (i * K0 + 16 * q) * 128, &tmap_a, kb * kKBLK,
-                          s * SR + i * p.R + 16 * q, &full[st]);
+                          ab_of(p.slot_map, s) * SR + i * p.R + 16 * q, &full[st]);
         }
         const int kcol = kb * kKBLK + c * 8;
         const bool cok = kcol < p.in;
@@ -745,14 +757,14 @@ cudaError_t dev_info(DevInfo** out) {
 template <typename P>
 cudaError_t launch_overlapped(void (*kern)(const CUtensorMap, const P), int grid, int threads,
                               size_t smem, cudaStream_t stream, const CUtensorMap& map,
-                              const P& p) {
+                              const P& p, bool allow_overlap = true) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3((unsigned)threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  if (launch_overlap_enabled()) {
+  if (allow_overlap && launch_overlap_enabled()) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
@@ -795,7 +807,8 @@ size_t sgmv_workspace_bytes(int T, int R, int S) {
 cudaError_t sgmv_shrink_launch(const void* x, const void* a, float* h, const int* ranks,
                                const int* token_order, const int* slot_indptr, int T, int in,
                                int slots, int R, int S, uint32_t* flags, cudaStream_t stream,
-                               const char** why, int ksplit_max, const float* scalings) {
+                               const char** why, int ksplit_max, const float* scalings,
+                               const SgmvGroups* groups) {
   if (in < kKBLK) {
     *why = "the SGMV shrink needs in_features >= 64";
     return cudaErrorNotSupported;
@@ -804,13 +817,18 @@ cudaError_t sgmv_shrink_launch(const void* x, const void* a, float* h, const int
   cudaError_t err = dev_info(&d);
   if (err != cudaSuccess) return err;
   CUtensorMap map;
-  err = make_map(&map, a, (uint64_t)in, (uint64_t)slots * S * R, kKBLK, 16,
+  const int ab_slots = groups != nullptr ? groups->ab_slots : slots;
+  err = make_map(&map, a, (uint64_t)in, (uint64_t)ab_slots * S * R, kKBLK, 16,
                  CU_TENSOR_MAP_SWIZZLE_128B, why);
   if (err != cudaSuccess) return err;
   ShrinkParams p = {};
   p.x = x; p.h = h; p.ranks = ranks; p.scalings = scalings; p.token_order = token_order;
   p.slot_indptr = slot_indptr; p.flags = flags; p.T = T; p.in = in; p.slots = slots; p.R = R;
   p.S = S;
+  if (groups != nullptr) {
+    p.seg_hi = groups->seg_hi;
+    p.slot_map = groups->slot_map;
+  }
   p.ksplit = min(ksplit_max, shrink_ksplit(T, slots, in, d->sms));
   p.kb_per_split = ceil_div_i(ceil_div_i(in, kKBLK), p.ksplit);
   p.h_split = (size_t)T * S * R;
@@ -823,7 +841,8 @@ cudaError_t sgmv_shrink_launch(const void* x, const void* a, float* h, const int
   }
   const int units = (slots + ceil_div_i(T, kTM)) * p.ksplit;
   const int grid = max(1, min(d->sms, units));
-  return launch_overlapped(sgmv_shrink_kernel, grid, kSgThreads, smem, stream, map, p);
+  return launch_overlapped(sgmv_shrink_kernel, grid, kSgThreads, smem, stream, map, p,
+                           groups == nullptr);
 }
 
 int sgmv_shrink_splits(int T, int slots, int in) {
@@ -836,7 +855,8 @@ cudaError_t sgmv_expand_launch(void* y, const float* h, int ksplit, const int* i
                                const void* b, const int* ranks, const float* scalings,
                                const int* token_order, const int* slot_indptr, int T, int vocab,
                                int slots, int R, int S, const int* slice_off, int out,
-                               uint32_t* flags, cudaStream_t stream, const char** why) {
+                               uint32_t* flags, cudaStream_t stream, const char** why,
+                               const SgmvGroups* groups) {
   DevInfo* d = nullptr;
   cudaError_t err = dev_info(&d);
   if (err != cudaSuccess) return err;
@@ -844,13 +864,18 @@ cudaError_t sgmv_expand_launch(void* y, const float* h, int ksplit, const int* i
   const CUtensorMapSwizzle swz = R == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : R == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                            : CU_TENSOR_MAP_SWIZZLE_32B;
-  err = make_map(&map, b, (uint64_t)R, (uint64_t)slots * out, (uint32_t)R, kBN, swz, why);
+  const int ab_slots = groups != nullptr ? groups->ab_slots : slots;
+  err = make_map(&map, b, (uint64_t)R, (uint64_t)ab_slots * out, (uint32_t)R, kBN, swz, why);
   if (err != cudaSuccess) return err;
   ExpandParams p = {};
   p.y = y; p.h = h; p.ksplit = ksplit; p.h_split = (size_t)T * S * R; p.ids = ids; p.a = a;
   p.ranks = ranks; p.scalings = scalings; p.token_order = token_order;
   p.slot_indptr = slot_indptr; p.flags = flags; p.T = T; p.vocab = vocab; p.slots = slots;
   p.R = R; p.S = S; p.out = out; p.span = 2 * R;
+  if (groups != nullptr) {
+    p.seg_hi = groups->seg_hi;
+    p.slot_map = groups->slot_map;
+  }
   int nchunk = 0;
   for (int i = 0; i <= LORA_MAX_SLICES; ++i) p.slice_off[i] = slice_off[i];
   for (int i = 0; i < S; ++i) {
@@ -868,7 +893,8 @@ cudaError_t sgmv_expand_launch(void* y, const float* h, int ksplit, const int* i
   }
   const long long units = (long long)(slots + ceil_div_i(T, kTM)) * nchunk;
   const int grid = (int)max(1LL, min((long long)d->sms, units));
-  return launch_overlapped(sgmv_expand_kernel, grid, kExThreads, smem, stream, map, p);
+  return launch_overlapped(sgmv_expand_kernel, grid, kExThreads, smem, stream, map, p,
+                           groups == nullptr);
 }
 
 }  // namespace lora

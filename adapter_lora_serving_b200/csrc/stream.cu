@@ -1,28 +1,30 @@
-// Embedding target (gather, then expand) in one launch over every SM: the
-// kernel lora_apply_embedding runs in the STREAM regime.
+// Streamed expand in one launch over every SM: the embedding target (the
+// kernel lora_apply_embedding runs in the STREAM regime) and the expand of a
+// computed h (the grouped MoE fold's expand).
 //
-//   h[t, i*R + r] = a[slot, i*R + r, ids[t]]        (r < rank; 0 for an id outside [0, vocab))
-//   y[t, off_i + j] = bf16_rne(y + scaling[slot] * sum_r h[t, i*R + r] * b[slot, off_i + j, r])
+//   embedding  h[t, i*R + r] = a[slot, i*R + r, ids[t]]   (r < rank; 0 for an id outside [0, vocab))
+//   computed   h[t, i*R + r] = sum over the partial buffers of h
+//   expand     y[t, off_i + j] = bf16_rne(y + scaling[slot] * sum_r h[t, i*R + r] * b[slot, off_i + j, r])
 //
 // Sources: mstar.engine.resources.lora.backend, LoraBackend.gather_shrink (the
 // one-hot shrink: a column of the slot's A per token id, nothing for an id
-// outside the vocabulary) and LoraBackend.apply_ with embedding=True (the
-// gathered h goes through the fused expand of expand_fused, over the slices
-// of out_slices laid out in order as in mstar.model.components.linear,
-// FusedColumnLinear).
+// outside the vocabulary), LoraBackend.expand_fused and apply_ with
+// embedding=True (the expand over the slices of out_slices laid out in order
+// as in mstar.model.components.linear, FusedColumnLinear);
+// spark_model/lora/expert_apply.rs, apply_expert_lora_sorted (the MoE fold's
+// expand over each (slot, expert) group of sorted rows).
 //
-// The work is the y read-modify-write: h is R bf16 values per token (exact:
-// they are elements of A) and B of all slots stays in L2.  So the kernel is
-// built around moving y at the HBM rate, with as few dependent memory round
-// trips before the stream starts as the data allows:
-//   * the output columns are cut into blocks of W = 512 / ksteps columns
-//     within one slice and the token positions into equal shares; CTA c takes
-//     block run c % bsplit and position share c / bsplit, so every CTA moves
-//     the same number of y bytes and a token's h is gathered by bsplit CTAs;
-//   * a CTA reads its share of token_order at once, next to the slot table,
-//     clips every live slot's segment to the share and cuts it into groups of
-//     16 positions (one MMA row tile); a unit is one (block, group) pair and
-//     the CTA walks its units block by block;
+// The work is the y read-modify-write: h is a few values per row and B of all
+// slots stays in L2.  So the kernel is built around moving y at the HBM rate,
+// with as few dependent memory round trips before the stream starts as the
+// data allows:
+//   * the positions of every slot (or group) that takes part are cut into
+//     row groups of 16 (one MMA row tile) and the output columns into blocks
+//     of W = 512 / ksteps columns within one slice; a unit is one (row group,
+//     block) pair; the units, row group by row group, are split into equal
+//     runs, one per CTA (one CTA per SM): the time a unit takes hardly depends
+//     on how many of its 16 rows are live, so equal counts balance the CTAs,
+//     and a row's h is read by one or two of them;
 //   * a producer warp bulk-copies a B block (W x R bf16, contiguous) into a
 //     ring of kStBBufs buffers whenever the (slot, block) changes; sixteen
 //     consumer warps take a 32-column chunk of the block each and keep their
@@ -32,10 +34,11 @@
 //     stream stays in flight in registers: bulk copies of single rows are too
 //     small to stream y at the HBM rate), runs m16n8k16 MMAs whose output
 //     columns are permuted so that its accumulators land on exactly those
-//     columns, and stores the 16 updated bytes of each row;
+//     columns, and stores the 16 updated bytes of each row; a computed fp32 h
+//     enters the MMAs as bf16 hi + lo (two MMAs, fp32 accumulate);
 //   * the planning, the tokens and the first B block are read before the
 //     wait on the preceding kernel (launch overlap); y, ids and h after it,
-//     the first units' y in flight while the ids and h are gathered.
+//     the first units' y in flight while h is gathered.
 // Waits on the B buffers' mbarriers are bounded (LORA_FLAG_TIMEOUT).
 #include <cuda_runtime.h>
 
@@ -86,52 +89,17 @@ LORA_DEV bool ring_ok(bool ok, int lane, int* abort_ring, uint32_t* pre_flags) {
   return true;
 }
 
-// The groups of one position share [plo, phi): slot s takes part when its
-// segment is valid (0 <= lo <= hi <= T), its rank is in (0, R] and its scaling
-// nonzero; its segment clipped to the share is cut into groups of kStRows.
-// Writes prefix[0..slots] (exclusive prefix of group counts) to shared memory
-// and returns the total.  Flags of bad segments and ranks are raised when
-// `report` is set.
-template <int NT>
-LORA_DEV int plan_share(const int* __restrict__ slot_indptr, const int* __restrict__ ranks,
-                        const float* __restrict__ scalings, int slots, int T, int R,
-                        long long plo, long long phi, int* prefix, int* scratch,
-                        uint32_t* flags, bool report) {
-  uint32_t bad = 0;
-  int carry = 0;
-  if (threadIdx.x == 0) prefix[0] = 0;
-  for (int base = 0; base < slots; base += NT) {
-    const int s = base + threadIdx.x;
-    int cnt = 0;
-    if (s < slots) {
-      const int lo = slot_indptr[s];
-      const int hi = slot_indptr[s + 1];
-      const int r = ranks[s];
-      const bool seg_ok = lo >= 0 && lo <= hi && hi <= T;
-      const bool rank_ok = r >= 0 && r <= R;
-      if (!seg_ok) bad |= LORA_FLAG_BAD_INDPTR;
-      if (!rank_ok) bad |= LORA_FLAG_BAD_RANK;
-      if (seg_ok && rank_ok && r > 0 && scalings[s] != 0.0f) {
-        const long long a = lo > plo ? lo : plo;
-        const long long b = hi < phi ? hi : phi;
-        if (b > a) cnt = (int)((b - a + kStRows - 1) / kStRows);
-      }
-    }
-    int tot;
-    const int inc = block_inclusive_scan<NT>(cnt, scratch, &tot);
-    if (s < slots) prefix[s + 1] = carry + inc;
-    carry += tot;
-  }
-  if (report) raise_flag(flags, bad);
-  __syncthreads();
-  return carry;
+// Segment end of slot (or group) s.
+LORA_DEV int seg_end(const StreamParams& p, int s) {
+  return p.seg_hi != nullptr ? p.seg_hi[s] : p.slot_indptr[s + 1];
 }
 
-template <int KS>
+// kH: h is computed (partial buffers); otherwise gathered from a by token id.
+template <int KS, bool kH>
 __global__ void __launch_bounds__(kStThreads, 1)
-    stream_embed_kernel(const __grid_constant__ StreamParams p) {
+    stream_kernel(const __grid_constant__ StreamParams p) {
   constexpr int Rp = KS * 16;
-  constexpr int D = KS >= 3 ? 2 : kStDepth;   // wide ranks: fewer units in flight
+  constexpr int D = (KS >= 3 || (kH && KS >= 2)) ? 2 : kStDepth;   // wide h: fewer units in flight
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t pre_flags;
   __shared__ int abort_ring;
@@ -140,13 +108,14 @@ __global__ void __launch_bounds__(kStThreads, 1)
   uint64_t* bempty = bfull + kStBBufs;
   int* prefix = reinterpret_cast<int*>(smem + p.off_prefix);
   int* scratch = reinterpret_cast<int*>(smem + p.off_scratch);
-  int* spec = reinterpret_cast<int*>(smem + p.off_spec);      // the share's token_order
+  int* spec = reinterpret_cast<int*>(smem + p.off_spec);      // token_order read ahead
   int* ctok = reinterpret_cast<int*>(smem + p.off_ctok);      // tokens of the window
-  int* cval = reinterpret_cast<int*>(smem + p.off_cval);      // token, or -1 (id outside)
+  int* cval = reinterpret_cast<int*>(smem + p.off_cval);      // token, or -1 (no h)
   int4* gmeta = reinterpret_cast<int4*>(smem + p.off_gmeta);  // slot, rank, scaling bits
   uint16_t* htab = reinterpret_cast<uint16_t*>(smem + p.off_htab);
   uint8_t* bbuf = smem + p.off_bbuf;
   const int SRp = p.S * Rp;
+  uint16_t* hlo = htab + (size_t)p.gtab * kStRows * SRp;     // kH: the bf16 remainders
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -161,51 +130,46 @@ __global__ void __launch_bounds__(kStThreads, 1)
     }
     fence_mbar_init();
   }
-  // this CTA's rectangle: blocks [b0, b1) x positions [plo, phi)
-  const int bsi = (int)(blockIdx.x % (unsigned)p.bsplit);
-  const int gsi = (int)(blockIdx.x / (unsigned)p.bsplit);
-  const int gsplit = (int)(gridDim.x / (unsigned)p.bsplit);
-  const int b0 = p.nblocks * bsi / p.bsplit;
-  const int b1 = p.nblocks * (bsi + 1) / p.bsplit;
-  const long long plo = (long long)p.T * gsi / gsplit;
-  const long long phi = (long long)p.T * (gsi + 1) / gsplit;
-  const int nshare = (int)(phi - plo);
-  const bool spec_ok = nshare <= kStSpec;
-  // the share's token_order, read next to the slot table (both addressing)
+  // token_order read ahead, next to the slot table: the positions this CTA
+  // takes when every position is live (the common layout); others are read
+  // when needed
+  const long long spec_lo = (long long)p.T * blockIdx.x / gridDim.x;
+  const long long spec_hi = (long long)p.T * (blockIdx.x + 1) / gridDim.x;
+  const int nspec = (int)((spec_hi - spec_lo) < kStSpec ? (spec_hi - spec_lo) : kStSpec);
   constexpr int kSv = (kStSpec + kStThreads - 1) / kStThreads;
   int sv[kSv];
 #pragma unroll
   for (int j = 0; j < kSv; ++j) {
     const int i = tid + j * kStThreads;
-    sv[j] = (spec_ok && i < nshare) ? p.token_order[plo + i] : -1;
+    sv[j] = i < nspec ? p.token_order[spec_lo + i] : -1;
   }
-  // plan_share synchronises the block before it reads or raises anything
-  const int planned = plan_share<kStThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
-                                             p.R, plo, phi, prefix, scratch, &pre_flags,
-                                             blockIdx.x == 0);
+  // plan_linear synchronises the block before it reads or raises anything
+  const int planned = plan_linear<kStThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
+                                              p.R, kStRows, prefix, scratch, &pre_flags,
+                                              blockIdx.x == 0, p.seg_hi);
 #pragma unroll
   for (int j = 0; j < kSv; ++j) {
     const int i = tid + j * kStThreads;
-    if (spec_ok && i < nshare) spec[i] = sv[j];
+    if (i < nspec) spec[i] = sv[j];
   }
-  // Disjoint segments give at most ceil(share/16) + slots groups; more means
-  // that segments overlap (tokens listed twice: the result is unspecified),
-  // and the surplus is dropped so that every count below stays in range.
-  const long long gcap = ((long long)nshare + kStRows - 1) / kStRows + p.slots;
-  const long long ng = (planned < 0 || planned > gcap) ? gcap : planned;
+  // Disjoint segments give at most ceil(T/16) + slots row groups; more means
+  // that segments overlap (positions listed twice: the result is
+  // unspecified), and the surplus is dropped so that every count below stays
+  // in range.
+  const long long gmax = ((long long)p.T + kStRows - 1) / kStRows + p.slots;
+  const long long ng = (planned < 0 || planned > gmax) ? gmax : planned;
+  // this CTA's run of units u = row_group * nblocks + block
+  const long long nu_all = ng * p.nblocks;
+  const long long u_lo = nu_all * blockIdx.x / gridDim.x;
+  const long long u_hi = nu_all * (blockIdx.x + 1) / gridDim.x;
   grid_dep_launch_dependents();
   __syncthreads();
 
   uint8_t* Y = static_cast<uint8_t*>(p.y);
   const uint16_t* A = static_cast<const uint16_t*>(p.a);
   const uint8_t* B = static_cast<const uint8_t*>(p.b);
-  // slices the CTA's blocks fall in: its h is gathered for those only
-  int sl_lo = 0, sl_hi = 0;
-  if (b1 > b0) {
-    while (sl_lo + 1 < p.S && b0 >= p.block_off[sl_lo + 1]) ++sl_lo;
-    sl_hi = sl_lo;
-    while (sl_hi + 1 < p.S && b1 - 1 >= p.block_off[sl_hi + 1]) ++sl_hi;
-  }
+  const int SR = p.S * p.R;
+  const int nb = p.nblocks;
 
   uint32_t bc = 0;                     // B blocks loaded (each role counts)
   int bkey_slot = -1, bkey_blk = -1;   // the B block in use (each role tracks it)
@@ -222,23 +186,30 @@ __global__ void __launch_bounds__(kStThreads, 1)
   const int brow = cw * 32 + 8 * (g8 >> 1) + (g8 & 1);
   uint2 bfr[4][KS];                    // B fragments of the block in use (consumers)
 
-  for (long long gw0 = 0; gw0 < ng && b1 > b0; gw0 += p.gtab) {
-    const int ngw = (int)((ng - gw0) < p.gtab ? (ng - gw0) : p.gtab);
+  const long long g_first = u_lo < u_hi ? u_lo / nb : 0;
+  const long long g_end = u_lo < u_hi ? (u_hi - 1) / nb + 1 : 0;
+  for (long long gw0 = g_first; gw0 < g_end; gw0 += p.gtab) {
+    const int ngw = (int)((g_end - gw0) < p.gtab ? (g_end - gw0) : p.gtab);
     const int nrows = ngw * kStRows;
+    // the window's units [wu0, wu1), row group by row group
+    const long long wu0 = u_lo > gw0 * nb ? u_lo : gw0 * nb;
+    const long long wu1 = u_hi < (gw0 + ngw) * nb ? u_hi : (gw0 + ngw) * nb;
+    const int nu = (int)(wu1 - wu0);
+    const int gi0 = (int)(wu0 / nb - gw0);
+    const int cb0 = (int)(wu0 % nb);
 
     // --- the window's tokens (addressing only: before the preceding kernel ends)
     for (int e = tid; e < nrows; e += kStThreads) {
       const int g = (int)(gw0 + e / kStRows);
       const int i = e % kStRows;
       const int s = find_segment(prefix, p.slots, g);
-      const int lo = p.slot_indptr[s];
-      const int hi = p.slot_indptr[s + 1];
-      const long long a = lo > plo ? lo : plo;
-      const long long b = hi < phi ? hi : phi;
-      const long long pos = a + (long long)(g - prefix[s]) * kStRows + i;
+      const long long lo = p.slot_indptr[s];
+      const long long hi = seg_end(p, s);
+      const long long pos = lo + (long long)(g - prefix[s]) * kStRows + i;
       int tok = -1;
-      if (pos >= a && pos < b) {
-        tok = spec_ok ? spec[pos - plo] : p.token_order[pos];
+      if (pos >= lo && pos < hi) {
+        tok = (pos >= spec_lo && pos < spec_lo + nspec) ? spec[pos - spec_lo]
+                                                        : p.token_order[pos];
         if (tok < 0 || tok >= p.T) {
           atomicOr(&pre_flags, LORA_FLAG_BAD_TOKEN);
           tok = -1;
@@ -253,16 +224,17 @@ __global__ void __launch_bounds__(kStThreads, 1)
     if (!waited) {
       // the first B block is an input: start it before the preceding kernel ends
       if (warp == 0) {
-        const int slot0 = gmeta[0].x;
+        const int slot0 = gmeta[gi0].x;
         if (lane == 0) {
           int sl, c0, ncols;
-          block_cols(p, b0, sl, c0, ncols);
+          block_cols(p, cb0, sl, c0, ncols);
           const uint32_t bb = (uint32_t)ncols * p.R * 2;
+          const int pair = p.slot_map != nullptr ? p.slot_map[slot0] : slot0;
           mbar_arrive_expect_tx(bfull, bb);
-          bulk_g2s(bbuf, B + ((size_t)slot0 * p.out + c0) * p.R * 2, bb, bfull);
+          bulk_g2s(bbuf, B + ((size_t)pair * p.out + c0) * p.R * 2, bb, bfull);
         }
         bkey_slot = slot0;
-        bkey_blk = b0;
+        bkey_blk = cb0;
         bc = 1;
       }
       grid_dep_wait();
@@ -271,44 +243,45 @@ __global__ void __launch_bounds__(kStThreads, 1)
 
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      bool stop = false;
-      for (int cb = b0; cb < b1 && !stop; ++cb) {
-        int sl, c0, ncols;
-        block_cols(p, cb, sl, c0, ncols);
-        for (int gi = 0; gi < ngw; ++gi) {
-          const int slot = gmeta[gi].x;
-          if (slot == bkey_slot && cb == bkey_blk) continue;
+      int gi = gi0, cb = cb0;
+      for (int u = 0; u < nu; ++u) {
+        const int slot = gmeta[gi].x;
+        if (slot != bkey_slot || cb != bkey_blk) {
+          int sl, c0, ncols;
+          block_cols(p, cb, sl, c0, ncols);
           // a new B block into the next buffer, once the consumers let it go
-          const int nb = (int)(bc % kStBBufs);
+          const int nbuf = (int)(bc % kStBBufs);
           const uint32_t kb = bc / kStBBufs;
-          const bool ok = kb > 0 ? ring_wait(bempty + nb, (kb - 1) & 1u, p.wait_ns) : true;
-          if (!ring_ok(ok, lane, &abort_ring, &pre_flags)) {
-            stop = true;
-            break;
-          }
+          const bool ok = kb > 0 ? ring_wait(bempty + nbuf, (kb - 1) & 1u, p.wait_ns) : true;
+          if (!ring_ok(ok, lane, &abort_ring, &pre_flags)) break;
           if (lane == 0) {
             const uint32_t bb = (uint32_t)ncols * p.R * 2;
-            mbar_arrive_expect_tx(bfull + nb, bb);
-            bulk_g2s(bbuf + (size_t)nb * p.bbytes, B + ((size_t)slot * p.out + c0) * p.R * 2, bb,
-                     bfull + nb);
+            const int pair = p.slot_map != nullptr ? p.slot_map[slot] : slot;
+            mbar_arrive_expect_tx(bfull + nbuf, bb);
+            bulk_g2s(bbuf + (size_t)nbuf * p.bbytes, B + ((size_t)pair * p.out + c0) * p.R * 2,
+                     bb, bfull + nbuf);
           }
           bkey_slot = slot;
           bkey_blk = cb;
           ++bc;
+        }
+        if (++cb == nb) {
+          cb = 0;
+          ++gi;
         }
       }
     } else {
       // ---------------------------------------------------------- consumers
       // units in order: block by block, the window's groups inside each block.
       // y of unit u + D is requested while unit u is computed; the first D
-      // units' y goes out before the ids are known (a row whose id turns out
-      // to be outside the vocabulary is read and left alone).
-      const int nu = (b1 - b0) * ngw;
+      // units' y goes out before h is read (a row that turns out to have no h
+      // -- an id outside the vocabulary -- is read and left alone).
       uint4 ya[D], yb[D];
-      int icb = b0, igi = 0;               // next unit to request
+      int icb = cb0, igi = gi0, ireq = 0;  // next unit to request
       auto request = [&](uint4& ra, uint4& rb) {
         ra = rb = make_uint4(0u, 0u, 0u, 0u);
-        if (icb >= b1) return;
+        if (ireq >= nu) return;
+        ++ireq;
         int sl, c0, ncols;
         block_cols(p, icb, sl, c0, ncols);
         if (cc < ncols) {
@@ -317,39 +290,52 @@ __global__ void __launch_bounds__(kStThreads, 1)
           if (tA >= 0) ra = *reinterpret_cast<const uint4*>(Y + ((size_t)tA * p.out + c0 + cc) * 2);
           if (tB >= 0) rb = *reinterpret_cast<const uint4*>(Y + ((size_t)tB * p.out + c0 + cc) * 2);
         }
-        if (++igi == ngw) {
-          igi = 0;
-          ++icb;
+        if (++icb == nb) {
+          icb = 0;
+          ++igi;
         }
       };
 #pragma unroll
       for (int j = 0; j < D; ++j) request(ya[j], yb[j]);
 
       const int ct = tid - 32;
-      // the rows' ids, then h for the slices of the CTA's blocks (zeros past
-      // the rank and for rows without a valid id)
-      const int ncolh = (sl_hi - sl_lo + 1) * Rp;
+      // h of the window's rows, every slice (zeros past the rank and for rows
+      // without h)
+      const int ncolh = SRp;
       for (int e = ct; e < nrows * ncolh; e += kStConsumers * 32) {
         const int row = e / ncolh;
         const int c = e - row * ncolh;
-        const int sl = sl_lo + c / Rp;
+        const int sl = c / Rp;
         const int r = c % Rp;
         const int4 gm = gmeta[row / kStRows];
         const int tok = ctok[row];
-        uint16_t v = 0;
-        bool valid = false;
-        if (tok >= 0) {
-          const int id = p.ids[tok];
-          valid = id >= 0 && id < p.vocab;
-          if (valid && r < gm.y)
-            v = A[((size_t)gm.x * p.S * p.R + (size_t)sl * p.R + r) * (size_t)p.vocab + id];
+        if (kH) {
+          float v = 0.0f;
+          if (tok >= 0 && r < gm.y) {
+            const float* hp = p.h + (size_t)tok * SR + sl * p.R + r;
+            for (int ks = 0; ks < p.ksplit; ++ks) v += hp[(size_t)ks * p.h_split];
+          }
+          const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+          htab[(size_t)row * SRp + sl * Rp + r] = *reinterpret_cast<const uint16_t*>(&hi);
+          hlo[(size_t)row * SRp + sl * Rp + r] = *reinterpret_cast<const uint16_t*>(&lo);
+          if (c == 0) cval[row] = tok;
+        } else {
+          uint16_t v = 0;
+          bool valid = false;
+          if (tok >= 0) {
+            const int id = p.ids[tok];
+            valid = id >= 0 && id < p.vocab;
+            if (valid && r < gm.y)
+              v = A[((size_t)gm.x * p.S * p.R + (size_t)sl * p.R + r) * (size_t)p.vocab + id];
+          }
+          htab[(size_t)row * SRp + sl * Rp + r] = v;
+          if (c == 0) cval[row] = valid ? tok : -1;
         }
-        htab[(size_t)row * SRp + sl * Rp + r] = v;
-        if (c == 0) cval[row] = valid ? tok : -1;
       }
       consumer_sync();
 
-      int pcb = b0, pgi = 0;               // unit being computed
+      int pcb = cb0, pgi = gi0;            // unit being computed
       bool stop = false;
       for (int u0 = 0; u0 < nu && !stop; u0 += D) {
 #pragma unroll
@@ -400,11 +386,11 @@ __global__ void __launch_bounds__(kStThreads, 1)
             // of each k-step) identically in h and B, which leaves the sum
             // unchanged
             uint2 hA[KS], hB[KS];
-            const uint16_t* hrow = htab + (size_t)rowA * SRp + sl * Rp + 4 * q;
+            const size_t hoff = (size_t)rowA * SRp + sl * Rp + 4 * q;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-              hA[ks] = *reinterpret_cast<const uint2*>(hrow + ks * 16);
-              hB[ks] = *reinterpret_cast<const uint2*>(hrow + 8 * SRp + ks * 16);
+              hA[ks] = *reinterpret_cast<const uint2*>(htab + hoff + ks * 16);
+              hB[ks] = *reinterpret_cast<const uint2*>(htab + hoff + 8 * SRp + ks * 16);
             }
             float d[4][4];
 #pragma unroll
@@ -415,6 +401,20 @@ __global__ void __launch_bounds__(kStThreads, 1)
               for (int ks = 0; ks < KS; ++ks)
                 mma_bf16_16816(d[jj], hA[ks].x, hB[ks].x, hA[ks].y, hB[ks].y, bfr[jj][ks].x,
                                bfr[jj][ks].y);
+            }
+            if (kH) {
+#pragma unroll
+              for (int ks = 0; ks < KS; ++ks) {
+                hA[ks] = *reinterpret_cast<const uint2*>(hlo + hoff + ks * 16);
+                hB[ks] = *reinterpret_cast<const uint2*>(hlo + hoff + 8 * SRp + ks * 16);
+              }
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks)
+                  mma_bf16_16816(d[jj], hA[ks].x, hB[ks].x, hA[ks].y, hB[ks].y, bfr[jj][ks].x,
+                                 bfr[jj][ks].y);
+              }
             }
             const float scal = __int_as_float(gm.z);
             const uint32_t yav[4] = {ya[j].x, ya[j].y, ya[j].z, ya[j].w};
@@ -434,9 +434,9 @@ __global__ void __launch_bounds__(kStThreads, 1)
               *reinterpret_cast<uint4*>(Y + ((size_t)tokB * p.out + c0 + cc) * 2) =
                   make_uint4(ob[0], ob[1], ob[2], ob[3]);
           }
-          if (++pgi == ngw) {
-            pgi = 0;
-            ++pcb;
+          if (++pcb == nb) {
+            pcb = 0;
+            ++pgi;
           }
           request(ya[j], yb[j]);     // unit u0 + j + D
         }
@@ -454,42 +454,54 @@ struct StreamDev {
   int dev;
   int sms;
   int max_smem;
-  unsigned attr_set;   // bit KS-1: the kernel's shared-memory limit is raised
+  unsigned attr_set;   // bit i: the shared-memory limit of kernel variant i is raised
 };
 std::mutex g_stream_mu;
 StreamDev g_stream_dev[64];
 int g_stream_n = 0;
 
-template <int KS>
-cudaError_t launch_ks(const StreamParams& p, int grid, cudaStream_t stream) {
+template <int KS, bool kH>
+cudaError_t launch_ks(const StreamParams& p, int grid, bool overlap, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(kStThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)p.smem;
   cfg.stream = stream;
-  if (launch_overlap_enabled()) {
+  if (overlap) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, stream_embed_kernel<KS>, p);
+  return cudaLaunchKernelEx(&cfg, stream_kernel<KS, kH>, p);
 }
 
-template <int KS>
+template <int KS, bool kH>
 cudaError_t raise_smem_limit(int bytes) {
-  return cudaFuncSetAttribute(stream_embed_kernel<KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(stream_kernel<KS, kH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               bytes);
+}
+
+cudaError_t raise_variant(int KS, bool kh, int bytes) {
+  switch (KS) {
+    case 1: return kh ? raise_smem_limit<1, true>(bytes) : raise_smem_limit<1, false>(bytes);
+    case 2: return kh ? raise_smem_limit<2, true>(bytes) : raise_smem_limit<2, false>(bytes);
+    case 3: return kh ? raise_smem_limit<3, true>(bytes) : raise_smem_limit<3, false>(bytes);
+    default: return kh ? raise_smem_limit<4, true>(bytes) : raise_smem_limit<4, false>(bytes);
+  }
 }
 
 }  // namespace
 
-cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char** why) {
+cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overlap,
+                          const char** why) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   const int KS = round_up_i(p.R, 16) / 16;
+  const bool kh = p.h != nullptr;
+  const unsigned bit = 1u << ((KS - 1) * 2 + (kh ? 1 : 0));
   StreamDev d = {-1, 0, 0, 0u};
   int slot = -1;
   {
@@ -509,15 +521,10 @@ cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char
     d.max_smem -= 256;
     d.dev = dev;
   }
-  if (!(d.attr_set & (1u << (KS - 1)))) {
-    switch (KS) {
-      case 1: err = raise_smem_limit<1>(d.max_smem); break;
-      case 2: err = raise_smem_limit<2>(d.max_smem); break;
-      case 3: err = raise_smem_limit<3>(d.max_smem); break;
-      default: err = raise_smem_limit<4>(d.max_smem); break;
-    }
+  if (!(d.attr_set & bit)) {
+    err = raise_variant(KS, kh, d.max_smem);
     if (err != cudaSuccess) return err;
-    d.attr_set |= 1u << (KS - 1);
+    d.attr_set |= bit;
     std::lock_guard<std::mutex> lk(g_stream_mu);
     if (slot >= 0) {
       g_stream_dev[slot] = d;
@@ -536,18 +543,15 @@ cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char
   p.nblocks = p.block_off[p.S];
 
   const int grid = d.sms;
-  // Two block runs when there are blocks enough and the grid is even (each
-  // token's h is then gathered by two CTAs), else one.
-  p.bsplit = (p.nblocks >= 4 && grid % 2 == 0) ? 2 : 1;
-  const int gsplit = grid / p.bsplit;
-  // groups of one share with disjoint segments: one window if they fit
-  const long long share = ((long long)p.T + gsplit - 1) / gsplit;
-  const long long per_cta = (share + kStRows - 1) / kStRows + p.slots;
-  p.gtab = (int)(per_cta < kStMaxGroups ? per_cta : kStMaxGroups);
+  // row groups one CTA's run touches with disjoint segments: one window if
+  // they fit
+  const long long gmax = ((long long)p.T + kStRows - 1) / kStRows + p.slots;
+  const long long per_cta = (gmax * p.nblocks + grid - 1) / grid / p.nblocks + 2;
+  const long long share = ((long long)p.T + grid - 1) / grid;
   const int nspec = (int)(share < kStSpec ? share : kStSpec);
 
-  // shared memory: barriers, plan prefix and scan scratch, the share's
-  // tokens, tables, B buffers
+  // shared memory: barriers, the group prefix, scan scratch, the tokens read
+  // ahead, tables (h twice when computed), B buffers
   int off = 2 * kStBBufs * 8;
   p.off_prefix = off;
   off += round_up_i((p.slots + 1) * 4, 16);
@@ -555,6 +559,16 @@ cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char
   off += round_up_i(kStThreads / 32 * 4, 16);
   p.off_spec = off;
   off += round_up_i(nspec * 4, 16);
+  // the tables take what is left beside the B buffers, at most kStMaxGroups
+  const int per_group = kStRows * 4 * 2 + 16 + (kh ? 2 : 1) * kStRows * p.S * Rp * 2;
+  const int room = d.max_smem - off - 64 - 128 - kStBBufs * p.bbytes;
+  long long gt = per_cta < kStMaxGroups ? per_cta : kStMaxGroups;
+  if (room / per_group < gt) gt = room / per_group;
+  if (gt < 1) {
+    *why = "shared memory of the streamed expand exceeds the device limit";
+    return cudaErrorInvalidConfiguration;
+  }
+  p.gtab = (int)gt;
   p.off_ctok = off;
   off += p.gtab * kStRows * 4;
   p.off_cval = off;
@@ -562,20 +576,25 @@ cudaError_t stream_embed_launch(StreamParams& p, cudaStream_t stream, const char
   p.off_gmeta = round_up_i(off, 16);
   off = p.off_gmeta + p.gtab * 16;
   p.off_htab = round_up_i(off, 16);
-  off = p.off_htab + p.gtab * kStRows * p.S * Rp * 2;
+  off = p.off_htab + (kh ? 2 : 1) * p.gtab * kStRows * p.S * Rp * 2;
   p.off_bbuf = round_up_i(off, 128);
   p.smem = p.off_bbuf + kStBBufs * p.bbytes;
   if (p.smem > d.max_smem) {
-    *why = "shared memory of the streamed embedding exceeds the device limit";
+    *why = "shared memory of the streamed expand exceeds the device limit";
     return cudaErrorInvalidConfiguration;
   }
   p.wait_ns = wait_limit_ns();
+  const bool overlap = allow_overlap && launch_overlap_enabled();
 
   switch (KS) {
-    case 1: return launch_ks<1>(p, grid, stream);
-    case 2: return launch_ks<2>(p, grid, stream);
-    case 3: return launch_ks<3>(p, grid, stream);
-    default: return launch_ks<4>(p, grid, stream);
+    case 1: return kh ? launch_ks<1, true>(p, grid, overlap, stream)
+                      : launch_ks<1, false>(p, grid, overlap, stream);
+    case 2: return kh ? launch_ks<2, true>(p, grid, overlap, stream)
+                      : launch_ks<2, false>(p, grid, overlap, stream);
+    case 3: return kh ? launch_ks<3, true>(p, grid, overlap, stream)
+                      : launch_ks<3, false>(p, grid, overlap, stream);
+    default: return kh ? launch_ks<4, true>(p, grid, overlap, stream)
+                       : launch_ks<4, false>(p, grid, overlap, stream);
   }
 }
 

@@ -153,10 +153,17 @@ class Workload:
         return d
 
     def _moe(self, m):
+        # the workspace selects the fold grouped by (slot, expert); it needs
+        # no initialisation
+        ws = self.L.lora_workspace_bytes(self.L.LORA_OP_EXPERT_APPLY, m.rows_cap, m.num_experts,
+                                         m.R, m.num_slices)
         return dict(m=m, x=self._bf16(m.x), y=self._bf16(m.y), a=self._bf16(m.a),
                     b=self._bf16(m.b), pair_index=self._i32(m.pair_index),
                     ranks=self._i32(m.ranks), scalings=self._f32(m.scalings),
-                    row_slot=self._i32(m.row_slot), offsets=self._i32(m.expert_offsets))
+                    row_slot=self._i32(m.row_slot), offsets=self._i32(m.expert_offsets),
+                    ws=self.torch.empty(max(ws, 16) // 4, dtype=self.torch.int32,
+                                        device="cuda") if ws else None,
+                    ws_bytes=ws)
 
     def _to_device(self, prob):
         if self.name == "moe_expert":
@@ -186,7 +193,8 @@ class Workload:
     @property
     def launches_per_step(self):
         if self.name == "moe_expert":
-            return 2
+            # per fold: the (slot, expert) grouping, the shrink and the expand
+            return 6 if self.sets[0][0]["ws"] is not None else 2
         p = self.host_sets[0]
         op = self.L.LORA_OP_APPLY_EMBEDDING if self.name == "embedding" else \
             self.L.LORA_OP_APPLY_LINEAR
@@ -204,7 +212,8 @@ class Workload:
                 L.lora_expert_apply(q["x"], q["y"], q["a"], q["b"], q["pair_index"], q["ranks"],
                                     q["scalings"], q["row_slot"], q["offsets"], m.rows_cap,
                                     m.n_in, m.num_experts, m.slots, m.num_pairs, m.R,
-                                    m.out_slices, stream=stream)
+                                    m.out_slices, workspace=q["ws"],
+                                    workspace_bytes=q["ws_bytes"], stream=stream)
             return
         p = d["p"]
         if self.name == "embedding":

@@ -231,7 +231,17 @@ LORA_API lora_status lora_apply_embedding(const int32_t* ids, void* y, const voi
  * pair_index [slots*num_experts] (-1 = not adapted); ranks, scalings [slots];
  * row_slot [rows_cap] (-1 = no adapter); expert_offsets [num_experts+1].
  * Planning happens on the device (no copy of expert_offsets to the host).
- * workspace may be NULL when lora_workspace_bytes(LORA_OP_EXPERT_APPLY, ...) is 0.
+ * Row blocks of different experts that overlap give an unspecified result for
+ * the shared rows.
+ * Without a workspace the fold runs one CTA per chunk of an expert's rows.
+ * With a workspace of lora_workspace_bytes(LORA_OP_EXPERT_APPLY, rows_cap,
+ * num_experts, R, num_slices, LORA_REGIME_AUTO) bytes (16-byte aligned, no
+ * initialisation needed; 0 when the shapes are outside the SGMV rule R in
+ * {16, 32, 64}, num_slices * R <= 128) and slots * num_experts <= 4096 and
+ * in_features >= 64, it is grouped by (slot, expert): a device pass sorts
+ * each adapted expert's rows by slot, then the tensor-core shrink and expand
+ * tile every (slot, expert) group like a slot's tokens (three launches).
+ * Otherwise the workspace is left unused.
  */
 LORA_API lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* a,
                               const void* b, const int32_t* pair_index, const int32_t* ranks,

@@ -128,12 +128,24 @@ class MoEDev:
         self.offsets = dev_i32(m.expert_offsets)
         self.flags = flags_buf()
 
-    def apply(self):
+    def apply(self, grouped=False, workspace=None):
+        """lora_expert_apply: without a workspace (the per-chunk BGMV kernel)
+        or, grouped=True, with a workspace of lora_workspace_bytes (the fold
+        grouped by (slot, expert) on the tensor-core kernels)."""
         m = self.m
+        ws_bytes = 0
+        if grouped:
+            ws_bytes = L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, m.rows_cap, m.num_experts,
+                                              m.R, m.num_slices)
+            assert ws_bytes > 0
+            if workspace is None:
+                t = torch()
+                workspace = t.empty(ws_bytes // 4 + 4, dtype=t.int32, device="cuda")
         L.lora_expert_apply(self.x, self.y, self.a, self.b, self.pair_index, self.ranks,
                             self.scalings, self.row_slot, self.offsets, m.rows_cap, m.n_in,
                             m.num_experts, m.slots, m.num_pairs, m.R, m.out_slices,
-                            err_flags=self.flags)
+                            workspace=workspace if grouped else None,
+                            workspace_bytes=ws_bytes, err_flags=self.flags)
 
 
 def assert_close(y_dev, y_ref, what=""):

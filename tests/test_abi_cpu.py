@@ -157,6 +157,14 @@ def test_host_queries(lib):
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_EMBEDDING, 64, 8, 72, 1) != \
         L.LORA_REGIME_STREAM
     assert L.lora_plan_tile(L.LORA_OP_APPLY_EMBEDDING, L.LORA_REGIME_STREAM) == 16
+    # the grouped expert fold: token_order, the group tables (4096 groups x 4
+    # ints), then four fp32 partial h buffers; nothing for the per-chunk kernel
+    rows, R, S = 16384, 16, 2
+    assert L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, rows, 128, R, S) == \
+        rows * 4 + 4 * 4096 * 4 + 4 * rows * R * S * 4
+    assert L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, rows, 128, R, S,
+                                  L.LORA_REGIME_BGMV) == 0
+    assert L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, rows, 128, 8, 1) == 0
 
 
 def test_wait_limit_setting_roundtrip(lib):
