@@ -13,7 +13,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "liblora_delta.so")
-SOURCES = ["api.cu", "bgmv.cu", "bgmv_split.cu", "stream.cu", "moe_group.cu", "plan.cu", "sgmv.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "bgmv.cu", "bgmv_split.cu", "stream.cu", "moe_group.cu", "group_shrink.cu", "plan.cu", "sgmv.cu", "noalloc.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -539,10 +539,18 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
     if (err != cudaSuccess) return cuda_fail(err, op, nullptr);
     const lora::SgmvGroups groups = {seg_hi, pair_index, num_pairs};
     const char* why = nullptr;
-    // live groups are about the pairs in use: split the shrink to fill the SMs
-    const int ks = lora::sgmv_shrink_splits(0, num_pairs < G ? num_pairs : G, in_features);
-    err = lora::sgmv_shrink_launch(x_sorted, a, hws, g_rank, tok, seg_lo, rows_cap, in_features,
-                                   G, R, num_slices, err_flags, s, &why, ks, g_scal, &groups);
+    int ks = 1;
+    if (lora::group_shrink_supported(num_slices, R, in_features)) {
+      // the groups are short: 16-row tiles, the features split into chunks
+      err = lora::group_shrink_launch(x_sorted, a, hws, tok, seg_lo, seg_hi, pair_index, g_rank,
+                                      g_scal, rows_cap, in_features, G, R, num_slices, &ks, s);
+    } else {
+      // live groups are about the pairs in use: split the shrink to fill the SMs
+      ks = lora::sgmv_shrink_splits(0, num_pairs < G ? num_pairs : G, in_features);
+      err = lora::sgmv_shrink_launch(x_sorted, a, hws, g_rank, tok, seg_lo, rows_cap,
+                                     in_features, G, R, num_slices, err_flags, s, &why, ks,
+                                     g_scal, &groups);
+    }
     if (err != cudaSuccess) return cuda_fail(err, op, why);
     // the expand: the groups are short (a few dozen rows), so their y rows are
     // streamed with 16-row MMA tiles rather than tiled by 128

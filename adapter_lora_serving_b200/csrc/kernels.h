@@ -342,6 +342,15 @@ inline bool stream_supported(int R) { return round_up_i(R, 16) <= kStMaxRp; }
 cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overlap,
                           const char** why);
 
+// Shrink of the grouped MoE fold over short segments (group_shrink.cu): row
+// groups of 16, the input features in chunks of 512 (at most 4), fp32 partial
+// h per chunk; S*R in {16, 32, 48, 64}.  *ksplit_out = the number of chunks.
+bool group_shrink_supported(int S, int R, int in);
+cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const int* token_order,
+                                const int* seg_lo, const int* seg_hi, const int* slot_map,
+                                const int* ranks, const float* scalings, int T, int in,
+                                int slots, int R, int S, int* ksplit_out, cudaStream_t stream);
+
 // The MoE fold grouped by (slot, expert) (moe_group.cu): per adapted expert,
 // its rows sorted by slot into token_order, group g = s * num_experts + e owning
 // [seg_lo[g], seg_hi[g]) with rank g_rank[g] and scaling g_scal[g].
