@@ -29,6 +29,7 @@ namespace lora {
 namespace {
 
 constexpr int kMgThreads = 256;
+constexpr int kMgCache = 4096;   // rows whose class is kept in shared memory between the passes
 
 struct MoeGroupParams {
   const int* expert_offsets;
@@ -46,7 +47,9 @@ struct MoeGroupParams {
 };
 
 // The row's group slot, or -1 when the row is left out (flags in *bad).
-LORA_DEV int classify_row(const MoeGroupParams& p, int e, int rho, uint32_t* bad) {
+// srank / sscal: the slots' ranks and scalings, read once into shared memory.
+LORA_DEV int classify_row(const MoeGroupParams& p, const int* srank, const float* sscal, int e,
+                          int rho, uint32_t* bad) {
   const int s = p.row_slot[rho];
   if (s == -1) return -1;
   if (s < -1 || s >= p.slots) {
@@ -59,12 +62,12 @@ LORA_DEV int classify_row(const MoeGroupParams& p, int e, int rho, uint32_t* bad
     *bad |= LORA_FLAG_BAD_PAIR;
     return -1;
   }
-  const int r = p.ranks[s];
+  const int r = srank[s];
   if (r < 0 || r > p.R) {
     *bad |= LORA_FLAG_BAD_RANK;
     return -1;
   }
-  if (r == 0 || p.scalings[s] == 0.0f) return -1;
+  if (r == 0 || sscal[s] == 0.0f) return -1;
   return s;
 }
 
@@ -72,6 +75,9 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
   extern __shared__ int sm[];
   int* cnt = sm;               // [slots] rows per slot
   int* cur = sm + p.slots;     // [slots] next position per slot
+  int* srank = cur + p.slots;  // [slots]
+  float* sscal = reinterpret_cast<float*>(srank + p.slots);   // [slots]
+  int* cls = reinterpret_cast<int*>(sscal + p.slots);         // [kMgCache] row classes
   __shared__ int scratch[kMgThreads / 32];
   __shared__ int adapted;
   __shared__ int dead_cur;
@@ -84,15 +90,22 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
     dead_cur = 0;
     bad_all = 0u;
   }
-  for (int s = tid; s < p.slots; s += kMgThreads) cnt[s] = 0;
+  // everything the classification needs besides the rows, in one round trip
+  const int off0 = p.expert_offsets[e];
+  const int off1 = p.expert_offsets[e + 1];
+  for (int s = tid; s < p.slots; s += kMgThreads) {
+    cnt[s] = 0;
+    srank[s] = p.ranks[s];
+    sscal[s] = p.scalings[s];
+  }
   __syncthreads();
   for (int s = tid; s < p.slots; s += kMgThreads)
     if (p.pair_index[(size_t)s * E + e] != -1) adapted = 1;
   __syncthreads();
   int start = 0, end = 0;
   if (adapted) {
-    start = p.expert_offsets[e];
-    end = p.expert_offsets[e + 1];
+    start = off0;
+    end = off1;
     if (start < 0 || end > p.rows_cap || end < start) {
       if (tid == 0) bad_all |= LORA_FLAG_BAD_OFFSETS;
       start = end = 0;
@@ -100,7 +113,8 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
   }
   uint32_t bad = 0;
   for (int rho = start + tid; rho < end; rho += kMgThreads) {
-    const int s = classify_row(p, e, rho, &bad);
+    const int s = classify_row(p, srank, sscal, e, rho, &bad);
+    if (rho - start < kMgCache) cls[rho - start] = s;
     if (s >= 0) atomicAdd(&cnt[s], 1);
   }
   if (bad) atomicOr(&bad_all, bad);
@@ -127,7 +141,8 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
   const int dead_lo = start + carry;
   for (int rho = start + tid; rho < end; rho += kMgThreads) {
     uint32_t unused = 0;
-    const int s = classify_row(p, e, rho, &unused);
+    const int s = rho - start < kMgCache ? cls[rho - start]
+                                         : classify_row(p, srank, sscal, e, rho, &unused);
     const int pos = s >= 0 ? atomicAdd(&cur[s], 1) : dead_lo + atomicAdd(&dead_cur, 1);
     p.token_order[pos] = rho;
   }
@@ -148,7 +163,12 @@ cudaError_t moe_group_launch(const int* expert_offsets, const int* pair_index, c
   p.seg_hi = seg_hi; p.g_rank = g_rank; p.g_scal = g_scal; p.flags = flags;
   p.rows_cap = rows_cap; p.num_experts = num_experts; p.slots = slots; p.num_pairs = num_pairs;
   p.R = R;
-  const size_t smem = (size_t)2 * slots * sizeof(int);
+  const size_t smem = (size_t)4 * slots * sizeof(int) + (size_t)kMgCache * sizeof(int);
+  if (smem > 48 * 1024) {
+    const cudaError_t err = cudaFuncSetAttribute(
+        moe_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+  }
   moe_group_kernel<<<num_experts, kMgThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
