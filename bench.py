@@ -559,7 +559,8 @@ KERNEL_SOURCES = {
     "bgmv_kernel": ["bgmv.cu", "common.cuh", "kernels.h", "expand_tile.cuh"],
     "sgmv_expand_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
     "sgmv_shrink_kernel": ["sgmv.cu", "sgmv.h", "tcgen05.cuh", "common.cuh", "kernels.h"],
-    "stream_embed_kernel": ["stream.cu", "common.cuh", "kernels.h", "expand_tile.cuh"],
+    "stream_kernel": ["stream.cu", "common.cuh", "kernels.h", "expand_tile.cuh"],
+    "group_shrink_kernel": ["group_shrink.cu", "common.cuh", "kernels.h"],
 }
 
 
