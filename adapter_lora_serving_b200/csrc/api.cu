@@ -89,28 +89,48 @@ lora_status check_ptrs(const char* op, std::initializer_list<std::pair<const voi
 
 bool bgmv_fits(int S, int R) { return S * lora::round_up_i(R, 16) <= lora::kMaxSRp; }
 
+constexpr long long kStreamLinearMaxWork = 1LL << 22;   // T * in_features AUTO streams up to
+
+bool stream_linear_fits(int T, int in_features, int S, int R) {
+  return lora::stream_supported(R) && lora::group_shrink_supported(S, R, in_features) &&
+         (long long)T * in_features <= kStreamLinearMaxWork;
+}
+
 int resolve(int regime, int op, int T, int slots, int R, int S, int in_features = 1 << 30) {
   if (regime == LORA_REGIME_BGMV || regime == LORA_REGIME_SGMV) return regime;
   if (regime == LORA_REGIME_BGMV_SPLIT)
     return op == LORA_OP_APPLY_LINEAR ? LORA_REGIME_BGMV_SPLIT : LORA_REGIME_BGMV;
   if (regime == LORA_REGIME_STREAM)
-    return op == LORA_OP_APPLY_EMBEDDING ? LORA_REGIME_STREAM : LORA_REGIME_BGMV;
+    return (op == LORA_OP_APPLY_EMBEDDING || op == LORA_OP_APPLY_LINEAR) ? LORA_REGIME_STREAM
+                                                                         : LORA_REGIME_BGMV;
   // the embedding: stream the output rows through shared memory
   if (op == LORA_OP_APPLY_EMBEDDING && lora::stream_supported(R)) return LORA_REGIME_STREAM;
   const bool needs_shrink = (op == LORA_OP_SHRINK || op == LORA_OP_APPLY_LINEAR);
   // Many tokens per slot on average: tensor-core tiles over slot segments.
   if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024 &&
-      (!needs_shrink || in_features >= 64))
+      (!needs_shrink || in_features >= 64)) {
+    // up to T * in_features = 2^22 the fused apply goes faster through the
+    // short-segment shrink and the streamed expand (measured: T = 1024..2048
+    // with in = 2048..4096 and narrow A, 1.3-1.7x; even at 2^23, behind from
+    // 2^24)
+    if (op == LORA_OP_APPLY_LINEAR && stream_linear_fits(T, in_features, S, R))
+      return LORA_REGIME_STREAM;
     return LORA_REGIME_SGMV;
+  }
   return LORA_REGIME_BGMV;
 }
 
 // Workspace bytes lora_apply_linear needs in regime `reg` (0: none).  SGMV:
 // the counter header (which it leaves alone), then the partial h buffers of
-// the split shrink.  BGMV_SPLIT: its counters and partials.  BGMV: none.
+// the split shrink.  BGMV_SPLIT: its counters and partials.  STREAM: the
+// counter header (which it leaves alone), then the partial h of every
+// 512-feature chunk.  BGMV: none.
 size_t apply_linear_need(int reg, int T, int in_features, int slots, int R, int S, int out) {
   if (T <= 0 || R <= 0 || S <= 0) return 0;
   if (reg == LORA_REGIME_SGMV) return lora::kWsCounterBytes + lora::sgmv_workspace_bytes(T, R, S);
+  if (reg == LORA_REGIME_STREAM)
+    return lora::kWsCounterBytes +
+           (size_t)lora::group_shrink_chunks(in_features) * T * S * R * sizeof(float);
   if (reg == LORA_REGIME_BGMV_SPLIT && lora::split_eligible(T, in_features, slots, R, S, out))
     return lora::split_workspace_bytes(T, slots, R, S);
   return 0;
@@ -169,7 +189,9 @@ int32_t lora_resolve_regime(int32_t op, int32_t T, int32_t slots, int32_t R, int
 
 int32_t lora_plan_tile(int32_t op, int32_t regime) {
   if (op == LORA_OP_EXPERT_APPLY) return lora::kTT;
-  if (op == LORA_OP_APPLY_EMBEDDING && regime == LORA_REGIME_STREAM) return lora::kStRows;
+  if ((op == LORA_OP_APPLY_EMBEDDING || op == LORA_OP_APPLY_LINEAR) &&
+      regime == LORA_REGIME_STREAM)
+    return lora::kStRows;
   if (regime == LORA_REGIME_SGMV) return lora::kSgmvTileM;
   if (op == LORA_OP_APPLY_LINEAR) return lora::kFusedTile;
   return lora::kTT;
@@ -185,8 +207,22 @@ size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R, int
   if (op != LORA_OP_APPLY_LINEAR || T <= 0 || R <= 0 || num_slices <= 0) return 0;
   const int reg = resolve(regime, op, T, slots, R, num_slices);
   // in_features and out are not known here: size for the largest the split
-  // kernel takes (it refuses larger ones)
-  return apply_linear_need(reg, T, lora::kSpMaxIn, slots, R, num_slices, lora::kSpMaxOut);
+  // and streamed kernels take (they refuse larger ones)
+  if (reg == LORA_REGIME_STREAM)
+    return apply_linear_need(reg, T, lora::kGsMaxIn, slots, R, num_slices, 0);
+  size_t need = apply_linear_need(reg, T, lora::kSpMaxIn, slots, R, num_slices, lora::kSpMaxOut);
+  if (regime == LORA_REGIME_AUTO && reg == LORA_REGIME_SGMV) {
+    // AUTO streams these shapes when in_features is small enough: the
+    // largest such in_features (a multiple of 8, at most 4096)
+    long long in_max = kStreamLinearMaxWork / T;
+    in_max = (in_max < lora::kGsMaxIn ? in_max : lora::kGsMaxIn) / 8 * 8;
+    if (in_max >= 64 && stream_linear_fits(T, (int)in_max, num_slices, R)) {
+      const size_t sneed =
+          apply_linear_need(LORA_REGIME_STREAM, T, (int)in_max, slots, R, num_slices, 0);
+      need = sneed > need ? sneed : need;
+    }
+  }
+  return need;
 }
 
 uint64_t lora_set_wait_limit_ns(uint64_t ns) { return lora::set_wait_limit_ns(ns); }
@@ -302,6 +338,35 @@ lora_status apply_linear_impl(const char* op, const void* x, void* y, const void
     return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
   const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, in_features);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (reg == LORA_REGIME_STREAM) {
+    // short-segment shrink into per-chunk partial h, then the streamed expand
+    if (!lora::stream_supported(R) || !lora::group_shrink_supported(num_slices, R, in_features))
+      return fail(LORA_ERR_UNSUPPORTED,
+                  "%s: the STREAM regime takes num_slices*R in {16, 32, 48, 64} and "
+                  "in_features <= %d", op, lora::kGsMaxIn);
+    const size_t need = apply_linear_need(reg, T, in_features, slots, R, num_slices, out);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(LORA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", op, need,
+                  workspace == nullptr ? (size_t)0 : workspace_bytes);
+    if (!aligned16(workspace))
+      return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
+    float* hws = reinterpret_cast<float*>(static_cast<char*>(workspace) + lora::kWsCounterBytes);
+    lora::StreamParams q = {};
+    const char* why = nullptr;
+    int ks = 1;
+    cudaError_t err = lora::group_shrink_launch(x, a, hws, token_order, slot_indptr, nullptr,
+                                                nullptr, ranks, scalings, T, in_features, slots,
+                                                R, num_slices, &ks, s, true);
+    if (err != cudaSuccess) return cuda_fail(err, op, nullptr);
+    q.h = hws; q.h_split = (size_t)T * num_slices * R; q.ksplit = ks;
+    q.y = y; q.b = b; q.ranks = ranks; q.scalings = scalings; q.token_order = token_order;
+    q.slot_indptr = slot_indptr; q.flags = err_flags;
+    q.T = T; q.vocab = 0; q.slots = slots; q.R = R; q.S = num_slices; q.out = out;
+    for (int i = 0; i <= LORA_MAX_SLICES; ++i) q.slice_off[i] = p.slice_off[i];
+    err = lora::stream_launch(q, s, true, &why);
+    if (err != cudaSuccess) return cuda_fail(err, op, why);
+    return ok();
+  }
   if (reg == LORA_REGIME_SGMV) {
     if (!lora::sgmv_supported(num_slices, R))
       return fail(LORA_ERR_UNSUPPORTED, "%s: %s", op, lora::kSgmvShapeRule);
@@ -543,7 +608,8 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
     if (lora::group_shrink_supported(num_slices, R, in_features)) {
       // the groups are short: 16-row tiles, the features split into chunks
       err = lora::group_shrink_launch(x_sorted, a, hws, tok, seg_lo, seg_hi, pair_index, g_rank,
-                                      g_scal, rows_cap, in_features, G, R, num_slices, &ks, s);
+                                      g_scal, rows_cap, in_features, G, R, num_slices, &ks, s,
+                                      false);
     } else {
       // live groups are about the pairs in use: split the shrink to fill the SMs
       ks = lora::sgmv_shrink_splits(0, num_pairs < G ? num_pairs : G, in_features);

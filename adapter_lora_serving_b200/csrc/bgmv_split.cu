@@ -141,11 +141,6 @@ LORA_DEV float4 ld_cg_f4(const float* p) {
                : "l"(p));
   return v;
 }
-LORA_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 LORA_DEV void prefetch_l2_line(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }

@@ -26,6 +26,13 @@ LORA_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// A load that acquires at GPU scope (pairs with a release or fence + atomic).
+LORA_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 LORA_DEV uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -268,12 +275,13 @@ LORA_DEV int block_inclusive_scan(int v, int* scratch, int* total) {
 // segments and ranks are raised when `report` is set.  The segment of slot s
 // is [slot_indptr[s], slot_indptr[s+1]), or [slot_indptr[s], seg_hi[s]) when
 // seg_hi is given (segments that need not abut, e.g. the MoE fold's
-// (slot, expert) groups).
+// (slot, expert) groups).  seg_out (optional, shared memory): every slot's
+// (lo, hi) as read.
 template <int NT>
 LORA_DEV int plan_linear(const int* __restrict__ slot_indptr, const int* __restrict__ ranks,
                          const float* __restrict__ scalings, int slots, int T, int R, int tile,
                          int* prefix, int* scratch, uint32_t* flags, bool report,
-                         const int* __restrict__ seg_hi = nullptr) {
+                         const int* __restrict__ seg_hi = nullptr, int2* seg_out = nullptr) {
   uint32_t bad = 0;
   int carry = 0;
   if (threadIdx.x == 0) prefix[0] = 0;
@@ -283,6 +291,7 @@ LORA_DEV int plan_linear(const int* __restrict__ slot_indptr, const int* __restr
     if (s < slots) {
       const int lo = slot_indptr[s];
       const int hi = seg_hi != nullptr ? seg_hi[s] : slot_indptr[s + 1];
+      if (seg_out != nullptr) seg_out[s] = make_int2(lo, hi);   // shared memory: the bounds as read
       const int r = ranks[s];
       const bool seg_ok = lo >= 0 && lo <= hi && hi <= T;
       const bool rank_ok = r >= 0 && r <= R;

@@ -8,7 +8,8 @@
 // spark_model/lora/expert_apply.rs, apply_expert_lora_sorted (the fold per
 // (slot, expert) group of sorted rows, each with its pair's A).
 //
-// Every group's positions [seg_lo, seg_hi) are cut into row groups of 16 and
+// Every group's positions [seg_lo, seg_hi) (or, without seg_hi, CSR by slot:
+// [seg_lo[s], seg_lo[s+1])) are cut into row groups of 16 and
 // the input features into chunks of 512; a unit is one (row group, chunk)
 // pair and the units, row group by row group, are split into equal runs, one
 // per CTA (one per SM).  All 16 warps of a CTA work on one unit: warp w takes
@@ -66,9 +67,11 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
   const int g8 = lane >> 2;
   const int q = lane & 3;
 
-  // the groups' row groups (the grouping pass validated segments and ranks)
+  // the groups' row groups (flags of bad segments and ranks are raised by the
+  // kernel that follows, which plans the same segments)
   const int planned = plan_linear<kGsThreads>(p.seg_lo, p.ranks, p.scalings, p.slots, p.T, p.R,
                                               kStRows, prefix, scratch, nullptr, false, p.seg_hi);
+  grid_dep_launch_dependents();
   const long long gmax = ((long long)p.T + kStRows - 1) / kStRows + p.slots;
   const long long ng = (planned < 0 || planned > gmax) ? gmax : planned;
   const long long nu = ng * p.nks;
@@ -83,7 +86,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
     const int kc = (int)(u - (long long)g * p.nks);
     const int s = find_segment(prefix, p.slots, g);
     const int lo = p.seg_lo[s];
-    const int hi = p.seg_hi[s];
+    const int hi = p.seg_hi != nullptr ? p.seg_hi[s] : p.seg_lo[s + 1];
     const int pair = p.slot_map != nullptr ? p.slot_map[s] : s;
     const int pa = lo + (g - prefix[s]) * kStRows + g8;
     const int pb = pa + 8;
@@ -152,6 +155,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
   };
 
   GsRegs<NT> r0, r1, r2;
+  grid_dep_wait();   // x (and the partial buffers) only after the preceding kernel
   if (u0 < u1) load(u0, r0);
   if (u0 + 1 < u1) load(u0 + 1, r1);
   for (long long u = u0; u < u1; u += 3) {
@@ -163,17 +167,27 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
   }
 }
 
+template <int NT>
+cudaError_t launch_nt(const cudaLaunchConfig_t& cfg, const GShrinkParams& p) {
+  const cudaError_t err = cudaFuncSetAttribute(
+      group_shrink_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      (int)cfg.dynamicSmemBytes);
+  if (err != cudaSuccess) return err;
+  return cudaLaunchKernelEx(&cfg, group_shrink_kernel<NT>, p);
+}
+
 }  // namespace
 
 bool group_shrink_supported(int S, int R, int in) {
   const int SR = S * R;
-  return (SR == 16 || SR == 32 || SR == 48 || SR == 64) && in <= 4 * 32 * kGsWarps;
+  return (SR == 16 || SR == 32 || SR == 48 || SR == 64) && in <= kGsMaxIn;
 }
 
 cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const int* token_order,
                                 const int* seg_lo, const int* seg_hi, const int* slot_map,
                                 const int* ranks, const float* scalings, int T, int in,
-                                int slots, int R, int S, int* ksplit_out, cudaStream_t stream) {
+                                int slots, int R, int S, int* ksplit_out, cudaStream_t stream,
+                                bool allow_overlap) {
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -182,32 +196,29 @@ cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const in
   p.x = x; p.a = a; p.h = h; p.h_split = (size_t)T * S * R; p.token_order = token_order;
   p.seg_lo = seg_lo; p.seg_hi = seg_hi; p.slot_map = slot_map; p.ranks = ranks;
   p.scalings = scalings; p.T = T; p.in = in; p.slots = slots; p.R = R; p.S = S;
-  p.nks = ceil_div_i(in, 32 * kGsWarps);
+  p.nks = group_shrink_chunks(in);
+  static_assert(32 * kGsWarps == 512, "one chunk is 512 features");
   *ksplit_out = p.nks;
   p.off_red = round_up_i((slots + 1 + kGsWarps) * 4, 16);
   const int SR = S * R;
   const size_t smem = (size_t)p.off_red + (size_t)kGsWarps * kStRows * SR * 4;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3((unsigned)sms, 1, 1);
+  cfg.blockDim = dim3(kGsThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  if (allow_overlap && launch_overlap_enabled()) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   switch (SR / 8) {
-    case 2:
-      err = cudaFuncSetAttribute(group_shrink_kernel<2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) group_shrink_kernel<2><<<sms, kGsThreads, smem, stream>>>(p);
-      break;
-    case 4:
-      err = cudaFuncSetAttribute(group_shrink_kernel<4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) group_shrink_kernel<4><<<sms, kGsThreads, smem, stream>>>(p);
-      break;
-    case 6:
-      err = cudaFuncSetAttribute(group_shrink_kernel<6>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) group_shrink_kernel<6><<<sms, kGsThreads, smem, stream>>>(p);
-      break;
-    default:
-      err = cudaFuncSetAttribute(group_shrink_kernel<8>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) group_shrink_kernel<8><<<sms, kGsThreads, smem, stream>>>(p);
-      break;
+    case 2: err = launch_nt<2>(cfg, p); break;
+    case 4: err = launch_nt<4>(cfg, p); break;
+    case 6: err = launch_nt<6>(cfg, p); break;
+    default: err = launch_nt<8>(cfg, p); break;
   }
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

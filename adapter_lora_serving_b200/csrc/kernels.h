@@ -330,7 +330,7 @@ struct StreamParams {
   int W;                               // columns per block at most
   int gtab;                            // groups per table window
   int bbytes;                          // bytes of one B buffer (W * R * 2)
-  int off_prefix, off_scratch, off_spec, off_ctok, off_cval, off_gmeta, off_htab;
+  int off_prefix, off_segs, off_scratch, off_spec, off_ctok, off_cval, off_gmeta, off_htab;
   int off_bbuf;
   int smem;
 };
@@ -342,14 +342,20 @@ inline bool stream_supported(int R) { return round_up_i(R, 16) <= kStMaxRp; }
 cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overlap,
                           const char** why);
 
-// Shrink of the grouped MoE fold over short segments (group_shrink.cu): row
-// groups of 16, the input features in chunks of 512 (at most 4), fp32 partial
-// h per chunk; S*R in {16, 32, 48, 64}.  *ksplit_out = the number of chunks.
+// Shrink over short segments (group_shrink.cu): row groups of 16, the input
+// features in chunks of 512 (at most 8), fp32 partial h per chunk; S*R in
+// {16, 32, 48, 64}.  Segments [seg_lo[s], seg_hi[s]), or CSR by slot
+// [seg_lo[s], seg_lo[s+1]) when seg_hi is null; A of pair slot_map[s] (s when
+// null).  *ksplit_out = the number of chunks.  allow_overlap: the
+// programmatic edge to the preceding kernel (x read and h written after it).
 bool group_shrink_supported(int S, int R, int in);
 cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const int* token_order,
                                 const int* seg_lo, const int* seg_hi, const int* slot_map,
                                 const int* ranks, const float* scalings, int T, int in,
-                                int slots, int R, int S, int* ksplit_out, cudaStream_t stream);
+                                int slots, int R, int S, int* ksplit_out, cudaStream_t stream,
+                                bool allow_overlap);
+constexpr int kGsMaxIn = 4096;
+inline int group_shrink_chunks(int in) { return ceil_div_i(in, 512); }
 
 // The MoE fold grouped by (slot, expert) (moe_group.cu): per adapted expert,
 // its rows sorted by slot into token_order, group g = s * num_experts + e owning

@@ -55,12 +55,13 @@ LORA_DEV void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers * 32) : "memory");
 }
 
-// Waits for a phase with the kernel's limit; false if it ran out.
-LORA_DEV bool ring_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+// Waits for a phase with the kernel's limit; false if it ran out or the CTA
+// has stopped (*abort set by another warp).
+LORA_DEV bool ring_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns, const int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > limit_ns) return false;
+    if (global_timer_ns() - t0 > limit_ns || *(const volatile int*)abort) return false;
   }
   return true;
 }
@@ -89,12 +90,8 @@ LORA_DEV bool ring_ok(bool ok, int lane, int* abort_ring, uint32_t* pre_flags) {
   return true;
 }
 
-// Segment end of slot (or group) s.
-LORA_DEV int seg_end(const StreamParams& p, int s) {
-  return p.seg_hi != nullptr ? p.seg_hi[s] : p.slot_indptr[s + 1];
-}
-
-// kH: h is computed (partial buffers); otherwise gathered from a by token id.
+// kH: h is summed from partial buffers an earlier kernel wrote; otherwise it
+// is gathered from a by token id.
 template <int KS, bool kH>
 __global__ void __launch_bounds__(kStThreads, 1)
     stream_kernel(const __grid_constant__ StreamParams p) {
@@ -107,6 +104,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
   uint64_t* bfull = reinterpret_cast<uint64_t*>(smem);
   uint64_t* bempty = bfull + kStBBufs;
   int* prefix = reinterpret_cast<int*>(smem + p.off_prefix);
+  int2* segs = reinterpret_cast<int2*>(smem + p.off_segs);      // every slot's (lo, hi)
   int* scratch = reinterpret_cast<int*>(smem + p.off_scratch);
   int* spec = reinterpret_cast<int*>(smem + p.off_spec);      // token_order read ahead
   int* ctok = reinterpret_cast<int*>(smem + p.off_ctok);      // tokens of the window
@@ -146,7 +144,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
   // plan_linear synchronises the block before it reads or raises anything
   const int planned = plan_linear<kStThreads>(p.slot_indptr, p.ranks, p.scalings, p.slots, p.T,
                                               p.R, kStRows, prefix, scratch, &pre_flags,
-                                              blockIdx.x == 0, p.seg_hi);
+                                              blockIdx.x == 0, p.seg_hi, segs);
 #pragma unroll
   for (int j = 0; j < kSv; ++j) {
     const int i = tid + j * kStThreads;
@@ -203,8 +201,9 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int g = (int)(gw0 + e / kStRows);
       const int i = e % kStRows;
       const int s = find_segment(prefix, p.slots, g);
-      const long long lo = p.slot_indptr[s];
-      const long long hi = seg_end(p, s);
+      const int2 sg = segs[s];
+      const long long lo = sg.x;
+      const long long hi = sg.y;
       const long long pos = lo + (long long)(g - prefix[s]) * kStRows + i;
       int tok = -1;
       if (pos >= lo && pos < hi) {
@@ -252,7 +251,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
           // a new B block into the next buffer, once the consumers let it go
           const int nbuf = (int)(bc % kStBBufs);
           const uint32_t kb = bc / kStBBufs;
-          const bool ok = kb > 0 ? ring_wait(bempty + nbuf, (kb - 1) & 1u, p.wait_ns) : true;
+          const bool ok =
+              kb > 0 ? ring_wait(bempty + nbuf, (kb - 1) & 1u, p.wait_ns, &abort_ring) : true;
           if (!ring_ok(ok, lane, &abort_ring, &pre_flags)) break;
           if (lane == 0) {
             const uint32_t bb = (uint32_t)ncols * p.R * 2;
@@ -302,25 +302,66 @@ __global__ void __launch_bounds__(kStThreads, 1)
       // h of the window's rows, every slice (zeros past the rank and for rows
       // without h)
       const int ncolh = SRp;
-      for (int e = ct; e < nrows * ncolh; e += kStConsumers * 32) {
-        const int row = e / ncolh;
-        const int c = e - row * ncolh;
-        const int sl = c / Rp;
-        const int r = c % Rp;
-        const int4 gm = gmeta[row / kStRows];
-        const int tok = ctok[row];
-        if (kH) {
-          float v = 0.0f;
-          if (tok >= 0 && r < gm.y) {
-            const float* hp = p.h + (size_t)tok * SR + sl * p.R + r;
-            for (int ks = 0; ks < p.ksplit; ++ks) v += hp[(size_t)ks * p.h_split];
+      const int nel = nrows * ncolh;
+      if (kH) {
+        // the sum of the partials in chunk order; two elements a thread and
+        // up to eight partials each in flight at once
+        constexpr int kStride = kStConsumers * 32;
+        for (int e0 = ct; e0 < nel; e0 += 2 * kStride) {
+          const float* hp[2];
+          int hrow[2], hcol[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int e = e0 + k * kStride;
+            hp[k] = nullptr;
+            hrow[k] = -1;
+            hcol[k] = 0;
+            if (e < nel) {
+              const int row = e / ncolh;
+              const int c = e - row * ncolh;
+              const int sl = c / Rp;
+              const int r = c % Rp;
+              const int tok = ctok[row];
+              hrow[k] = row;
+              hcol[k] = sl * Rp + r;
+              if (tok >= 0 && r < gmeta[row / kStRows].y)
+                hp[k] = p.h + (size_t)tok * SR + sl * p.R + r;
+              if (c == 0) cval[row] = tok;
+            }
           }
-          const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-          htab[(size_t)row * SRp + sl * Rp + r] = *reinterpret_cast<const uint16_t*>(&hi);
-          hlo[(size_t)row * SRp + sl * Rp + r] = *reinterpret_cast<const uint16_t*>(&lo);
-          if (c == 0) cval[row] = tok;
-        } else {
+          float v[2] = {0.0f, 0.0f};
+          for (int k0 = 0; k0 < p.ksplit; k0 += 8) {
+            float t[2][8];
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                t[k][j] = (hp[k] != nullptr && k0 + j < p.ksplit)
+                              ? __ldcg(hp[k] + (size_t)(k0 + j) * p.h_split)
+                              : 0.0f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (k0 + j < p.ksplit) v[k] += t[k][j];
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            if (hrow[k] < 0) continue;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v[k]);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(v[k] - __bfloat162float(hi));
+            htab[(size_t)hrow[k] * SRp + hcol[k]] = *reinterpret_cast<const uint16_t*>(&hi);
+            hlo[(size_t)hrow[k] * SRp + hcol[k]] = *reinterpret_cast<const uint16_t*>(&lo);
+          }
+        }
+      } else {
+        for (int e = ct; e < nel; e += kStConsumers * 32) {
+          const int row = e / ncolh;
+          const int c = e - row * ncolh;
+          const int sl = c / Rp;
+          const int r = c % Rp;
+          const int4 gm = gmeta[row / kStRows];
+          const int tok = ctok[row];
           uint16_t v = 0;
           bool valid = false;
           if (tok >= 0) {
@@ -348,7 +389,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
             // the next B block: its fragments into registers, then free the buffer
             const int nb = (int)(bc % kStBBufs);
             const uint32_t kb = bc / kStBBufs;
-            if (!ring_ok(ring_wait(bfull + nb, kb & 1u, p.wait_ns), lane, &abort_ring,
+            if (!ring_ok(ring_wait(bfull + nb, kb & 1u, p.wait_ns, &abort_ring), lane, &abort_ring,
                          &pre_flags)) {
               stop = true;
               break;
@@ -461,7 +502,11 @@ StreamDev g_stream_dev[64];
 int g_stream_n = 0;
 
 template <int KS, bool kH>
-cudaError_t launch_ks(const StreamParams& p, int grid, bool overlap, cudaStream_t stream) {
+cudaError_t launch_variant(const StreamParams& p, int grid, bool overlap, cudaStream_t stream,
+                           bool raise_only, int smem_limit) {
+  if (raise_only)
+    return cudaFuncSetAttribute(stream_kernel<KS, kH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem_limit);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
@@ -477,18 +522,19 @@ cudaError_t launch_ks(const StreamParams& p, int grid, bool overlap, cudaStream_
   return cudaLaunchKernelEx(&cfg, stream_kernel<KS, kH>, p);
 }
 
-template <int KS, bool kH>
-cudaError_t raise_smem_limit(int bytes) {
-  return cudaFuncSetAttribute(stream_kernel<KS, kH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              bytes);
-}
-
-cudaError_t raise_variant(int KS, bool kh, int bytes) {
+// The kernel variant of (KS, kh): launched, or (raise_only) its shared-memory
+// limit raised.
+cudaError_t dispatch(int KS, bool kh, const StreamParams& p, int grid, bool overlap,
+                     cudaStream_t stream, bool raise_only, int smem_limit) {
   switch (KS) {
-    case 1: return kh ? raise_smem_limit<1, true>(bytes) : raise_smem_limit<1, false>(bytes);
-    case 2: return kh ? raise_smem_limit<2, true>(bytes) : raise_smem_limit<2, false>(bytes);
-    case 3: return kh ? raise_smem_limit<3, true>(bytes) : raise_smem_limit<3, false>(bytes);
-    default: return kh ? raise_smem_limit<4, true>(bytes) : raise_smem_limit<4, false>(bytes);
+    case 1: return kh ? launch_variant<1, true>(p, grid, overlap, stream, raise_only, smem_limit)
+                      : launch_variant<1, false>(p, grid, overlap, stream, raise_only, smem_limit);
+    case 2: return kh ? launch_variant<2, true>(p, grid, overlap, stream, raise_only, smem_limit)
+                      : launch_variant<2, false>(p, grid, overlap, stream, raise_only, smem_limit);
+    case 3: return kh ? launch_variant<3, true>(p, grid, overlap, stream, raise_only, smem_limit)
+                      : launch_variant<3, false>(p, grid, overlap, stream, raise_only, smem_limit);
+    default: return kh ? launch_variant<4, true>(p, grid, overlap, stream, raise_only, smem_limit)
+                       : launch_variant<4, false>(p, grid, overlap, stream, raise_only, smem_limit);
   }
 }
 
@@ -522,7 +568,7 @@ cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overl
     d.dev = dev;
   }
   if (!(d.attr_set & bit)) {
-    err = raise_variant(KS, kh, d.max_smem);
+    err = dispatch(KS, kh, p, 0, false, stream, true, d.max_smem);
     if (err != cudaSuccess) return err;
     d.attr_set |= bit;
     std::lock_guard<std::mutex> lk(g_stream_mu);
@@ -555,6 +601,8 @@ cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overl
   int off = 2 * kStBBufs * 8;
   p.off_prefix = off;
   off += round_up_i((p.slots + 1) * 4, 16);
+  p.off_segs = off;
+  off += round_up_i(p.slots * 8, 16);
   p.off_scratch = off;
   off += round_up_i(kStThreads / 32 * 4, 16);
   p.off_spec = off;
@@ -586,16 +634,7 @@ cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overl
   p.wait_ns = wait_limit_ns();
   const bool overlap = allow_overlap && launch_overlap_enabled();
 
-  switch (KS) {
-    case 1: return kh ? launch_ks<1, true>(p, grid, overlap, stream)
-                      : launch_ks<1, false>(p, grid, overlap, stream);
-    case 2: return kh ? launch_ks<2, true>(p, grid, overlap, stream)
-                      : launch_ks<2, false>(p, grid, overlap, stream);
-    case 3: return kh ? launch_ks<3, true>(p, grid, overlap, stream)
-                      : launch_ks<3, false>(p, grid, overlap, stream);
-    default: return kh ? launch_ks<4, true>(p, grid, overlap, stream)
-                       : launch_ks<4, false>(p, grid, overlap, stream);
-  }
+  return dispatch(KS, kh, p, grid, overlap, stream, false, 0);
 }
 
 }  // namespace lora

@@ -112,10 +112,11 @@ def moe_cost(m):
 class Workload:
     """Rotating device input sets and the library call of one step."""
 
-    def __init__(self, name, n_sets, seed0, torch, L):
+    def __init__(self, name, n_sets, seed0, torch, L, regime=None):
         self.name = name
         self.torch = torch
         self.L = L
+        self.regime = L.LORA_REGIME_AUTO if regime is None else regime
         self.sets = []
         self.host_sets = []
         gen = W.WORKLOADS[name]
@@ -145,7 +146,7 @@ class Workload:
         if p.ids is not None:
             d["ids"] = self._i32(p.ids)
         ws = self.L.lora_workspace_bytes(self.L.LORA_OP_APPLY_LINEAR, p.T, p.slots, p.R,
-                                         p.num_slices)
+                                         p.num_slices, self.regime)
         d["ws_bytes"] = ws
         # zeroed once: the library keeps its counter header zeroed between calls
         d["ws"] = self.torch.zeros(max(ws, 16) // 4, dtype=self.torch.float32,
@@ -198,8 +199,9 @@ class Workload:
         p = self.host_sets[0]
         op = self.L.LORA_OP_APPLY_EMBEDDING if self.name == "embedding" else \
             self.L.LORA_OP_APPLY_LINEAR
-        reg = self.L.lora_resolve_regime(op, p.T, p.slots, p.R, p.num_slices)
-        if reg == self.L.LORA_REGIME_SGMV and self.name != "embedding":
+        reg = self.L.lora_resolve_regime(op, p.T, p.slots, p.R, p.num_slices) \
+            if self.regime == self.L.LORA_REGIME_AUTO else self.regime
+        if reg in (self.L.LORA_REGIME_SGMV, self.L.LORA_REGIME_STREAM) and self.name != "embedding":
             return 2
         return 1
 
@@ -219,18 +221,18 @@ class Workload:
         if self.name == "embedding":
             L.lora_apply_embedding(d["ids"], d["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                                    d["token_order"], d["slot_indptr"], p.T, p.n_in, p.slots, p.R,
-                                   p.out_slices, stream=stream)
+                                   p.out_slices, regime=self.regime, stream=stream)
             return
         if self.name == "moe_router":
             L.lora_apply_router(d["x"], d["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                                 d["token_order"], d["slot_indptr"], p.T, p.n_in, p.slots, p.R,
-                                p.out, workspace=d["ws"], workspace_bytes=d["ws_bytes"],
-                                stream=stream)
+                                p.out, regime=self.regime, workspace=d["ws"],
+                                workspace_bytes=d["ws_bytes"], stream=stream)
             return
         L.lora_apply_linear(d["x"], d["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                             d["token_order"], d["slot_indptr"], p.T, p.n_in, p.slots, p.R,
-                            p.out_slices, workspace=d["ws"], workspace_bytes=d["ws_bytes"],
-                            stream=stream)
+                            p.out_slices, regime=self.regime, workspace=d["ws"],
+                            workspace_bytes=d["ws_bytes"], stream=stream)
 
 
 def n_sets_for(name):
@@ -430,15 +432,16 @@ def time_e2e(torch, wl, steps):
         if wl.name == "embedding":
             L.lora_apply_embedding(dev["ids"], dev["y"], d["a"], d["b"], d["ranks"],
                                    d["scalings"], dev["token_order"], dev["slot_indptr"], p.T,
-                                   p.n_in, p.slots, p.R, p.out_slices)
+                                   p.n_in, p.slots, p.R, p.out_slices, regime=wl.regime)
         elif wl.name == "moe_router":
             L.lora_apply_router(dev["x"], dev["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                                 dev["token_order"], dev["slot_indptr"], p.T, p.n_in, p.slots,
-                                p.R, p.out, workspace=d["ws"], workspace_bytes=d["ws_bytes"])
+                                p.R, p.out, regime=wl.regime, workspace=d["ws"],
+                                workspace_bytes=d["ws_bytes"])
         else:
             L.lora_apply_linear(dev["x"], dev["y"], d["a"], d["b"], d["ranks"], d["scalings"],
                                 dev["token_order"], dev["slot_indptr"], p.T, p.n_in, p.slots,
-                                p.R, p.out_slices, workspace=d["ws"],
+                                p.R, p.out_slices, regime=wl.regime, workspace=d["ws"],
                                 workspace_bytes=d["ws_bytes"])
         out.copy_(dev["y"], non_blocking=True)
 
@@ -615,6 +618,9 @@ def main():
                     help="launch each step's kernel only after the previous one has finished")
     ap.add_argument("--profile", action="store_true",
                     help="timed steps only (no e2e, CPU baseline or table): for ncu captures")
+    ap.add_argument("--regime", default="auto",
+                    choices=["auto", "bgmv", "sgmv", "bgmv_split", "stream"],
+                    help="the headline workload's regime (the other rows of the table: auto)")
     ap.add_argument("--clock-window", type=float, default=0.4,
                     help="seconds of untimed replay of the step, under the clock sampler, "
                          "directly before the timed steps")
@@ -644,7 +650,8 @@ def main():
 
     name = args.workload
     nset = n_sets_for(name)
-    wl = Workload(name, nset, rank_seed0(rank, nset), torch, L)
+    regime = getattr(L, "LORA_REGIME_" + args.regime.upper())
+    wl = Workload(name, nset, rank_seed0(rank, nset), torch, L, regime)
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     except Exception:

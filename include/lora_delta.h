@@ -89,9 +89,10 @@ typedef enum {
 #define LORA_REGIME_SGMV 2   /* many tokens per slot: tcgen05/TMEM tiles over slot segments */
 #define LORA_REGIME_BGMV_SPLIT 3  /* few tokens per slot, the work split by bytes over every SM
                                      (lora_apply_linear only; needs a zeroed workspace) */
-#define LORA_REGIME_STREAM 4 /* output rows streamed through shared memory by bulk copies, the
-                                delta from warp MMAs (lora_apply_embedding only; AUTO's choice
-                                there) */
+#define LORA_REGIME_STREAM 4 /* output rows streamed in 16-row groups by every SM, the delta
+                                from warp MMAs (lora_apply_embedding: AUTO's choice there;
+                                lora_apply_linear: after a short-segment shrink, AUTO's
+                                choice for mid-size batches) */
 
 #define LORA_MAX_SLICES 8
 #define LORA_MAX_SLOTS 4096
@@ -140,6 +141,14 @@ LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const i
  *     of one slot), h kept in distributed shared memory; no workspace.
  *   SGMV: a tensor-core shrink writes fp32 partial h (one buffer per split of
  *     the input features) into the workspace and the expand sums them.
+ *   STREAM: two launches over every SM: a shrink over 16-row groups of each
+ *     slot's tokens writes fp32 partial h per 512 input features into the
+ *     workspace, then the streamed expand sums them (rows in 16-row groups,
+ *     y by 16-byte loads and stores).  Takes num_slices*R in {16, 32, 48,
+ *     64}, roundup(R, 16) <= 64 and in_features <= 4096 (else
+ *     LORA_ERR_UNSUPPORTED).  AUTO takes it where it would take SGMV and
+ *     T * in_features <= 2^22 with those shapes (lora_resolve_regime, which
+ *     does not know in_features, answers SGMV there).
  *   BGMV_SPLIT (only when asked for): one launch over every SM; the shrink is
  *     cut along the input features and the expand along the output columns
  *     into equal shares, and fp32 partial h pass through the workspace (each
@@ -149,7 +158,8 @@ LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const i
  *     LORA_ERR_UNSUPPORTED.
  * workspace must hold lora_workspace_bytes(LORA_OP_APPLY_LINEAR, T, slots, R,
  * num_slices, regime) bytes and be 16-byte aligned (may be NULL when that is
- * 0).  Its first 4096 bytes are the BGMV_SPLIT counters: a workspace that
+ * 0); for AUTO that covers whichever regime the call resolves to, STREAM
+ * included.  Its first 4096 bytes are the BGMV_SPLIT counters: a workspace that
  * BGMV_SPLIT calls use must be ZEROED before its first use (e.g. one
  * cudaMemsetAsync); every call leaves them zeroed again (zero them again after a
  * call that raised LORA_FLAG_TIMEOUT).  The rest needs no initialisation.

@@ -157,6 +157,19 @@ def test_host_queries(lib):
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_EMBEDDING, 64, 8, 72, 1) != \
         L.LORA_REGIME_STREAM
     assert L.lora_plan_tile(L.LORA_OP_APPLY_EMBEDDING, L.LORA_REGIME_STREAM) == 16
+    assert L.lora_plan_tile(L.LORA_OP_APPLY_LINEAR, L.LORA_REGIME_STREAM) == 16
+    # the fused apply in STREAM: the counter header, then one fp32 partial h
+    # per 512 input features, sized for in_features = 4096
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
+                                  L.LORA_REGIME_STREAM) == 4096 + 8 * 256 * 3 * 16 * 4
+    # AUTO would stream T = 1024 with in_features up to 4096 (T * in <= 2^22):
+    # its workspace covers that as well as SGMV's four partial buffers
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 1024, 4, 16, 1) == \
+        4096 + 8 * 1024 * 16 * 4
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 8192, 4, 16, 1) == \
+        4096 + 4 * 8192 * 16 * 4
+    # lora_resolve_regime does not know in_features: SGMV's shapes answer SGMV
+    assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 2048, 4, 16, 1) == L.LORA_REGIME_SGMV
     # the grouped expert fold: token_order, the group tables (4096 groups x 4
     # ints), then four fp32 partial h buffers; nothing for the per-chunk kernel
     rows, R, S = 16384, 16, 2
