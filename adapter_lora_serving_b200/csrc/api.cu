@@ -89,11 +89,21 @@ lora_status check_ptrs(const char* op, std::initializer_list<std::pair<const voi
 
 bool bgmv_fits(int S, int R) { return S * lora::round_up_i(R, 16) <= lora::kMaxSRp; }
 
-constexpr long long kStreamLinearMaxWork = 1LL << 22;   // T * in_features AUTO streams up to
+// The fused apply's shapes AUTO streams (given the workspace): measured on
+// the B200 against SGMV and BGMV with S*R <= 64, the short-segment shrink and
+// the streamed expand are ahead from T = 512 (BGMV ahead below) up to
+// T * in_features = 2^25 and T * out = 2^26 (SGMV ahead beyond), and at
+// T = 16384 SGMV is ahead again.
+constexpr int kStreamLinearMinT = 512;
+constexpr int kStreamLinearMaxT = 8192;
+constexpr long long kStreamLinearMaxIn = 1LL << 25;    // T * in_features
+constexpr long long kStreamLinearMaxOut = 1LL << 26;   // T * out
 
-bool stream_linear_fits(int T, int in_features, int S, int R) {
+bool stream_linear_fits(int T, int in_features, int out, int S, int R) {
   return lora::stream_supported(R) && lora::group_shrink_supported(S, R, in_features) &&
-         (long long)T * in_features <= kStreamLinearMaxWork;
+         T >= kStreamLinearMinT && T <= kStreamLinearMaxT &&
+         (long long)T * in_features <= kStreamLinearMaxIn &&
+         (long long)T * out <= kStreamLinearMaxOut;
 }
 
 int resolve(int regime, int op, int T, int slots, int R, int S, int in_features = 1 << 30) {
@@ -108,15 +118,8 @@ int resolve(int regime, int op, int T, int slots, int R, int S, int in_features 
   const bool needs_shrink = (op == LORA_OP_SHRINK || op == LORA_OP_APPLY_LINEAR);
   // Many tokens per slot on average: tensor-core tiles over slot segments.
   if (lora::sgmv_supported(S, R) && slots > 0 && (long long)T >= 64LL * slots && T >= 1024 &&
-      (!needs_shrink || in_features >= 64)) {
-    // up to T * in_features = 2^22 the fused apply goes faster through the
-    // short-segment shrink and the streamed expand (measured: T = 1024..2048
-    // with in = 2048..4096 and narrow A, 1.3-1.7x; even at 2^23, behind from
-    // 2^24)
-    if (op == LORA_OP_APPLY_LINEAR && stream_linear_fits(T, in_features, S, R))
-      return LORA_REGIME_STREAM;
+      (!needs_shrink || in_features >= 64))
     return LORA_REGIME_SGMV;
-  }
   return LORA_REGIME_BGMV;
 }
 
@@ -137,13 +140,27 @@ size_t apply_linear_need(int reg, int T, int in_features, int slots, int R, int 
 }
 
 // Workspace of the grouped expert fold: token_order [rows_cap], the group
-// tables (seg_lo, seg_hi, g_rank, g_scal; kMoeMaxGroups each), then the SGMV
-// partial h buffers.  0 when the shapes are not the SGMV kernels'.
+// tables (seg_lo, seg_hi, g_rank, g_scal; kMoeMaxGroups each), then the
+// partial h buffers (the short-segment shrink's eight, or the SGMV shrink's
+// four).  0 when the shapes are not the SGMV kernels'.
 size_t expert_group_need(int rows_cap, int R, int S) {
   if (rows_cap <= 0 || !lora::sgmv_supported(S, R)) return 0;
   const size_t tok = ((size_t)rows_cap * 4 + 255) / 256 * 256;
   const size_t tables = (size_t)4 * lora::kMoeMaxGroups * 4;
-  return tok + tables + lora::sgmv_workspace_bytes(rows_cap, R, S);
+  const size_t parts = (size_t)lora::kGsMaxParts * rows_cap * R * S * sizeof(float);
+  const size_t sgmv = lora::sgmv_workspace_bytes(rows_cap, R, S);
+  return tok + tables + (parts > sgmv ? parts : sgmv);
+}
+
+// lora_apply_linear's regime: resolve()'s, except that AUTO streams the
+// shapes stream_linear_fits() takes when ws_bytes holds the STREAM workspace.
+int resolve_linear(int regime, int T, int slots, int R, int S, int in_features, int out,
+                   size_t ws_bytes) {
+  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, S, in_features);
+  if (regime == LORA_REGIME_AUTO && stream_linear_fits(T, in_features, out, S, R) &&
+      ws_bytes >= apply_linear_need(LORA_REGIME_STREAM, T, in_features, slots, R, S, out))
+    return LORA_REGIME_STREAM;
+  return reg;
 }
 
 int linear_items_bound(int T, int slots, int tile) {
@@ -157,8 +174,8 @@ namespace lora {
 // Lets other entry points of the library report through lora_last_error().
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,
-                              int out) {
-  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, S, in_features);
+                              int out, size_t ws_bytes) {
+  const int reg = resolve_linear(regime, T, slots, R, S, in_features, out, ws_bytes);
   return apply_linear_need(reg, T, in_features, slots, R, S, out);
 }
 }  // namespace lora
@@ -211,12 +228,12 @@ size_t lora_workspace_bytes(int32_t op, int32_t T, int32_t slots, int32_t R, int
   if (reg == LORA_REGIME_STREAM)
     return apply_linear_need(reg, T, lora::kGsMaxIn, slots, R, num_slices, 0);
   size_t need = apply_linear_need(reg, T, lora::kSpMaxIn, slots, R, num_slices, lora::kSpMaxOut);
-  if (regime == LORA_REGIME_AUTO && reg == LORA_REGIME_SGMV) {
-    // AUTO streams these shapes when in_features is small enough: the
-    // largest such in_features (a multiple of 8, at most 4096)
-    long long in_max = kStreamLinearMaxWork / T;
+  if (regime == LORA_REGIME_AUTO) {
+    // AUTO streams these shapes when in_features is small enough (and is
+    // given the workspace): room for the largest such in_features
+    long long in_max = kStreamLinearMaxIn / T;
     in_max = (in_max < lora::kGsMaxIn ? in_max : lora::kGsMaxIn) / 8 * 8;
-    if (in_max >= 64 && stream_linear_fits(T, (int)in_max, num_slices, R)) {
+    if (in_max >= 8 && stream_linear_fits(T, (int)in_max, 8, num_slices, R)) {
       const size_t sneed =
           apply_linear_need(LORA_REGIME_STREAM, T, (int)in_max, slots, R, num_slices, 0);
       need = sneed > need ? sneed : need;
@@ -336,7 +353,8 @@ lora_status apply_linear_impl(const char* op, const void* x, void* y, const void
   if (st != LORA_OK) return st;
   if (err_flags != nullptr && !aligned4(err_flags))
     return fail(LORA_ERR_INVALID, "%s: err_flags is not 4-byte aligned", op);
-  const int reg = resolve(regime, LORA_OP_APPLY_LINEAR, T, slots, R, num_slices, in_features);
+  const int reg = resolve_linear(regime, T, slots, R, num_slices, in_features, out,
+                                 workspace != nullptr ? workspace_bytes : 0);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (reg == LORA_REGIME_STREAM) {
     // short-segment shrink into per-chunk partial h, then the streamed expand

@@ -1,6 +1,7 @@
 // Shrink over short segments: the (slot, expert) groups of the grouped MoE
-// fold hold a few dozen rows each, so the rows are taken 16 at a time (one
-// m16n8k16 row tile) instead of in 128-row tensor-core tiles.
+// fold hold a few dozen rows each, and so do the slots of a mid-size batch,
+// so the rows are taken 16 at a time (one m16n8k16 row tile) instead of in
+// 128-row tensor-core tiles.
 //
 //   h[kc][t, i*R + r] = sum over the features k of chunk kc of x[t, k] * a[pair, i*R + r, k]
 //
@@ -9,17 +10,23 @@
 // (slot, expert) group of sorted rows, each with its pair's A).
 //
 // Every group's positions [seg_lo, seg_hi) (or, without seg_hi, CSR by slot:
-// [seg_lo[s], seg_lo[s+1])) are cut into row groups of 16 and
-// the input features into chunks of 512; a unit is one (row group, chunk)
-// pair and the units, row group by row group, are split into equal runs, one
-// per CTA (one per SM).  All 16 warps of a CTA work on one unit: warp w takes
-// 32 of the chunk's features (two k-steps), loads its x and A fragments with
-// 8-byte loads (the k index permuted identically in both, thread q holding
-// k = 4q..4q+3 of each k-step, which leaves the sum unchanged) and runs the
-// MMAs for all S*R columns; the 16 partial tiles are summed in a fixed order
-// through shared memory and the chunk's fp32 h is written to its partial
-// buffer.  Each thread keeps the loads of the next two units in flight.
-// Columns past a group's rank are computed and never read.
+// [seg_lo[s], seg_lo[s+1])) are cut into row groups of 16 and the input
+// features into at most 8 chunks of 256 << k features; a unit is one (row
+// group, chunk) pair and the units, row group by row group, are split into
+// equal runs, one per CTA (one per SM).
+//
+// The 16 warps of a CTA form teams of TS warps (TS chosen per CTA from its
+// unit count: the fewer the units, the larger the teams); a team takes every
+// (16 / TS)-th unit of the run and its warps split the unit's 32-feature
+// sub-steps round robin.  A warp streams its sub-steps without a break, unit
+// after unit: thread q loads features 8q..8q+7 of the sub-step for its two x
+// rows and its A rows with one 16-byte load each, the next sub-steps' loads in
+// flight, and feeds 8q..8q+3 to one k-step MMA and 8q+4..8q+7 to the other
+// (the same permutation of k in both operands leaves the sum unchanged).  At
+// the end of a unit a one-warp team stores its fp32 tile straight to the
+// chunk's partial buffer; a larger team sums its warps' tiles in warp order
+// through shared memory first.  Columns past a group's rank are computed and
+// never read.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -43,24 +50,42 @@ struct GShrinkParams {
   const int* ranks;
   const float* scalings;
   int T, in, slots, R, S, nks;
-  int off_red;               // shared-memory offset of the reduction tiles
+  int chunk;                 // features per chunk (256 << k)
+  int off_segs, off_red;     // shared-memory offsets
 };
 
-// The fragments one thread loads for one unit.
+// One sub-step's fragments of one thread: 8 features of rows g and g + 8 of
+// x, and of A rows 8j + g.
 template <int NT>
-struct GsRegs {
-  uint2 xa[2], xb[2];     // rows g and g + 8, k-steps 0 and 1
-  uint2 af[NT][2];        // A rows 8j + g, k-steps 0 and 1
-  int ta, tb;             // the two rows' tokens (-1: none)
+struct GsSet {
+  uint4 xa, xb;
+  uint4 af[NT];
+};
+
+LORA_DEV uint4 ldg16(const uint8_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+LORA_DEV void team_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Sub-steps in flight per warp (what the registers hold beside the tile).
+template <int NT>
+struct GsSets {
+  static constexpr int value = NT <= 2 ? 4 : NT <= 4 ? 3 : NT <= 6 ? 2 : 1;
 };
 
 template <int NT>
 __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShrinkParams p) {
   constexpr int SR = NT * 8;
+  constexpr int SRP = SR + 8;     // padded tile row: conflict-free 8-byte stores
+  constexpr int NSET = GsSets<NT>::value;
   extern __shared__ __align__(16) uint8_t smem[];
-  int* prefix = reinterpret_cast<int*>(smem);     // [slots + 1]
-  int* scratch = prefix + p.slots + 1;            // [kGsWarps]
-  float* red = reinterpret_cast<float*>(smem + p.off_red);   // [kGsWarps][16][SR]
+  int* prefix = reinterpret_cast<int*>(smem);                    // [slots + 1]
+  int* scratch = prefix + p.slots + 1;                           // [kGsWarps]
+  int2* segs = reinterpret_cast<int2*>(smem + p.off_segs);       // [slots]
+  float* red = reinterpret_cast<float*>(smem + p.off_red);       // [kGsWarps][16][SRP]
+  __shared__ int utok[kGsWarps][NSET][kStRows + 1];   // a unit's 16 row tokens and its chunk
+  __shared__ int rtok[kGsWarps][kStRows];             // a team's 16 row tokens
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -70,100 +95,174 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
   // the groups' row groups (flags of bad segments and ranks are raised by the
   // kernel that follows, which plans the same segments)
   const int planned = plan_linear<kGsThreads>(p.seg_lo, p.ranks, p.scalings, p.slots, p.T, p.R,
-                                              kStRows, prefix, scratch, nullptr, false, p.seg_hi);
+                                              kStRows, prefix, scratch, nullptr, false, p.seg_hi,
+                                              segs);
   grid_dep_launch_dependents();
   const long long gmax = ((long long)p.T + kStRows - 1) / kStRows + p.slots;
   const long long ng = (planned < 0 || planned > gmax) ? gmax : planned;
   const long long nu = ng * p.nks;
   const long long u0 = nu * blockIdx.x / gridDim.x;
   const long long u1 = nu * (blockIdx.x + 1) / gridDim.x;
+  const int cnt = (int)(u1 - u0);
+  const int nsub = p.chunk / 32;
+
+  // team size: the fewest sub-step times for this CTA's units, a team's
+  // reduction counted as two (ties: the smaller team)
+  int TS = 1;
+  {
+    long long best = -1;
+    for (int ts = 1; ts <= kGsWarps && ts <= nsub; ts *= 2) {
+      const int teams = kGsWarps / ts;
+      const long long cost =
+          (long long)((cnt + teams - 1) / teams) * (nsub / ts + (ts > 1 ? 2 : 0));
+      if (best < 0 || cost < best) {
+        best = cost;
+        TS = ts;
+      }
+    }
+  }
+  const int nteams = kGsWarps / TS;
+  const int tm = warp / TS;
+  const int wt = warp - tm * TS;
+  const int nun = cnt > tm ? (cnt - tm + nteams - 1) / nteams : 0;   // this team's units
+  const int per = nsub / TS;                                          // sub-steps per unit and warp
+  const int K = nun * per;
+
   const uint8_t* X = static_cast<const uint8_t*>(p.x);
   const uint8_t* A = static_cast<const uint8_t*>(p.a);
 
-  // unit u: row group u / nks, feature chunk u % nks; this thread's loads
-  auto load = [&](long long u, GsRegs<NT>& r) {
+  // unit r of this team: its first position (row g8 of this lane), segment
+  // end, pair and chunk
+  auto unit_pos = [&](int r, int& pa, int& hi, int& pair, int& kc) {
+    const long long u = u0 + tm + (long long)r * nteams;
     const int g = (int)(u / p.nks);
-    const int kc = (int)(u - (long long)g * p.nks);
+    kc = (int)(u - (long long)g * p.nks);
     const int s = find_segment(prefix, p.slots, g);
-    const int lo = p.seg_lo[s];
-    const int hi = p.seg_hi != nullptr ? p.seg_hi[s] : p.seg_lo[s + 1];
-    const int pair = p.slot_map != nullptr ? p.slot_map[s] : s;
-    const int pa = lo + (g - prefix[s]) * kStRows + g8;
-    const int pb = pa + 8;
-    r.ta = pa < hi ? p.token_order[pa] : -1;
-    r.tb = pb < hi ? p.token_order[pb] : -1;
-    if (r.ta < 0 || r.ta >= p.T) r.ta = -1;
-    if (r.tb < 0 || r.tb >= p.T) r.tb = -1;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      const int k0 = kc * (32 * kGsWarps) + warp * 32 + ks * 16 + 4 * q;
-      const bool kin = k0 < p.in;
-      r.xa[ks] = (kin && r.ta >= 0)
-                     ? *reinterpret_cast<const uint2*>(X + ((size_t)r.ta * p.in + k0) * 2)
-                     : make_uint2(0u, 0u);
-      r.xb[ks] = (kin && r.tb >= 0)
-                     ? *reinterpret_cast<const uint2*>(X + ((size_t)r.tb * p.in + k0) * 2)
-                     : make_uint2(0u, 0u);
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-        r.af[j][ks] = kin ? *reinterpret_cast<const uint2*>(
-                                A + (((size_t)pair * SR + 8 * j + g8) * p.in + k0) * 2)
-                          : make_uint2(0u, 0u);
+    const int2 sg = segs[s];
+    pair = p.slot_map != nullptr ? p.slot_map[s] : s;
+    pa = sg.x + (g - prefix[s]) * kStRows + g8;
+    hi = sg.y;
+  };
+  // the unit the load cursor is in (its tokens, pair, feature range) and the
+  // raw tokens of the next one, read while this one loads
+  int lr = -1, l_ta = -1, l_tb = -1, l_pair = 0, l_k0 = 0, l_k1 = 0;
+  int n_ta = -1, n_tb = -1;
+  auto read_ahead = [&](int r) {
+    n_ta = n_tb = -1;
+    if (r < nun) {
+      int pa, hi, pair, kc;
+      unit_pos(r, pa, hi, pair, kc);
+      if (pa < hi) n_ta = p.token_order[pa];
+      if (pa + 8 < hi) n_tb = p.token_order[pa + 8];
     }
   };
-  // one unit: MMAs on r, the loads of unit un into rn (two units ahead), the
-  // warp's partial tile and the rows' tokens into shared memory, then the sum
-  // over the warps in a fixed order into the chunk's partial buffer
-  int* rowtok = scratch;   // the plan is done: its scan scratch holds the 16 row tokens
-  auto step = [&](long long u, GsRegs<NT>& r, long long un, GsRegs<NT>& rn) {
-    float d[NT][4];
+  read_ahead(0);
+  auto issue = [&](int k, GsSet<NT>& st) {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    if (k >= K) {
+      st.xa = st.xb = z;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
+      for (int j = 0; j < NT; ++j) st.af[j] = z;
+      return;
+    }
+    const int r = k / per;
+    if (r != lr) {
+      // units are entered in order, so the read-ahead holds this one's tokens
+      int pa, hi, pair, kc;
+      unit_pos(r, pa, hi, pair, kc);
+      lr = r;
+      l_ta = (n_ta < 0 || n_ta >= p.T) ? -1 : n_ta;
+      l_tb = (n_tb < 0 || n_tb >= p.T) ? -1 : n_tb;
+      l_pair = pair;
+      l_k0 = kc * p.chunk;
+      l_k1 = min(p.in, l_k0 + p.chunk);
+      if (q == 0) {
+        utok[warp][r % NSET][g8] = l_ta;
+        utok[warp][r % NSET][g8 + 8] = l_tb;
+      }
+      if (lane == 0) utok[warp][r % NSET][kStRows] = kc;
+      read_ahead(r + 1);
+    }
+    const int j = wt + (k - r * per) * TS;
+    const int k0 = l_k0 + 32 * j + 8 * q;
+    const bool kin = k0 < l_k1;   // in is a multiple of 8: the 8 features are all in or all out
+    st.xa = (kin && l_ta >= 0) ? ldg16(X + ((size_t)l_ta * p.in + k0) * 2) : z;
+    st.xb = (kin && l_tb >= 0) ? ldg16(X + ((size_t)l_tb * p.in + k0) * 2) : z;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) d[j][e] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks)
-        mma_bf16_16816(d[j], r.xa[ks].x, r.xb[ks].x, r.xa[ks].y, r.xb[ks].y, r.af[j][ks].x,
-                       r.af[j][ks].y);
-    }
-    float* rw = red + (size_t)warp * kStRows * SR;
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      rw[g8 * SR + 8 * j + 2 * q] = d[j][0];
-      rw[g8 * SR + 8 * j + 2 * q + 1] = d[j][1];
-      rw[(g8 + 8) * SR + 8 * j + 2 * q] = d[j][2];
-      rw[(g8 + 8) * SR + 8 * j + 2 * q + 1] = d[j][3];
-    }
-    if (warp == 0 && q == 0) {
-      rowtok[g8] = r.ta;
-      rowtok[g8 + 8] = r.tb;
-    }
-    const int kc = (int)(u % p.nks);
-    if (un < u1) load(un, rn);
-    __syncthreads();
-    for (int idx = tid; idx < kStRows * SR; idx += kGsThreads) {
-      const int row = idx / SR;
-      const int col = idx - row * SR;
-      const int t = rowtok[row];
-      if (t < 0) continue;
-      float v = 0.f;
-#pragma unroll 4
-      for (int w = 0; w < kGsWarps; ++w) v += red[((size_t)w * kStRows + row) * SR + col];
-      p.h[(size_t)kc * p.h_split + (size_t)t * SR + col] = v;
-    }
-    __syncthreads();
+    for (int jj = 0; jj < NT; ++jj)
+      st.af[jj] = kin ? ldg16(A + (((size_t)l_pair * SR + 8 * jj + g8) * p.in + k0) * 2) : z;
   };
 
-  GsRegs<NT> r0, r1, r2;
+  float d[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
+  // the end of unit r: its tile to the chunk's partial buffer
+  auto finish = [&](int r) {
+    __syncwarp();
+    const int* ut = utok[warp][r % NSET];
+    const int ra = ut[g8];
+    const int rb = ut[g8 + 8];
+    float* hk = p.h + (size_t)ut[kStRows] * p.h_split;
+    if (TS == 1) {
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        if (ra >= 0)
+          __stcg(reinterpret_cast<float2*>(hk + (size_t)ra * SR + 8 * j + 2 * q),
+                 make_float2(d[j][0], d[j][1]));
+        if (rb >= 0)
+          __stcg(reinterpret_cast<float2*>(hk + (size_t)rb * SR + 8 * j + 2 * q),
+                 make_float2(d[j][2], d[j][3]));
+      }
+    } else {
+      float* rw = red + (size_t)warp * kStRows * SRP;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        *reinterpret_cast<float2*>(rw + g8 * SRP + 8 * j + 2 * q) = make_float2(d[j][0], d[j][1]);
+        *reinterpret_cast<float2*>(rw + (g8 + 8) * SRP + 8 * j + 2 * q) =
+            make_float2(d[j][2], d[j][3]);
+      }
+      if (wt == 0 && q == 0) {
+        rtok[tm][g8] = ra;
+        rtok[tm][g8 + 8] = rb;
+      }
+      team_sync(1 + tm, TS * 32);
+      const float* rt = red + (size_t)tm * TS * kStRows * SRP;
+      for (int idx = wt * 32 + lane; idx < kStRows * SR; idx += TS * 32) {
+        const int row = idx / SR;
+        const int col = idx - row * SR;
+        const int t = rtok[tm][row];
+        if (t < 0) continue;
+        float v = 0.f;
+        for (int w = 0; w < TS; ++w) v += rt[((size_t)w * kStRows + row) * SRP + col];
+        __stcg(hk + (size_t)t * SR + col, v);
+      }
+      team_sync(1 + tm, TS * 32);
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
+  };
+
   grid_dep_wait();   // x (and the partial buffers) only after the preceding kernel
-  if (u0 < u1) load(u0, r0);
-  if (u0 + 1 < u1) load(u0 + 1, r1);
-  for (long long u = u0; u < u1; u += 3) {
-    step(u, r0, u + 2, r2);
-    if (u + 1 >= u1) break;
-    step(u + 1, r1, u + 3, r0);
-    if (u + 2 >= u1) break;
-    step(u + 2, r2, u + 4, r1);
+  GsSet<NT> set[NSET];
+#pragma unroll
+  for (int b = 0; b < NSET; ++b) issue(b, set[b]);
+  for (int k = 0; k < K; k += NSET) {
+#pragma unroll
+    for (int b = 0; b < NSET; ++b) {
+      const int kk = k + b;
+      if (kk < K) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          mma_bf16_16816(d[j], set[b].xa.x, set[b].xb.x, set[b].xa.y, set[b].xb.y,
+                         set[b].af[j].x, set[b].af[j].y);
+          mma_bf16_16816(d[j], set[b].xa.z, set[b].xb.z, set[b].xa.w, set[b].xb.w,
+                         set[b].af[j].z, set[b].af[j].w);
+        }
+        // a unit is finished before the load cursor may reuse its token slot
+        if ((kk + 1) % per == 0) finish(kk / per);
+        issue(kk + NSET, set[b]);
+      }
+    }
   }
 }
 
@@ -178,9 +277,17 @@ cudaError_t launch_nt(const cudaLaunchConfig_t& cfg, const GShrinkParams& p) {
 
 }  // namespace
 
+int group_shrink_chunk(int in) {
+  int c = 256;
+  while ((long long)c * kGsMaxParts < in) c *= 2;
+  return c;
+}
+
+int group_shrink_chunks(int in) { return ceil_div_i(in, group_shrink_chunk(in)); }
+
 bool group_shrink_supported(int S, int R, int in) {
   const int SR = S * R;
-  return (SR == 16 || SR == 32 || SR == 48 || SR == 64) && in <= kGsMaxIn;
+  return (SR == 16 || SR == 32 || SR == 48 || SR == 64) && in >= 8 && in <= kGsMaxIn;
 }
 
 cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const int* token_order,
@@ -196,12 +303,13 @@ cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const in
   p.x = x; p.a = a; p.h = h; p.h_split = (size_t)T * S * R; p.token_order = token_order;
   p.seg_lo = seg_lo; p.seg_hi = seg_hi; p.slot_map = slot_map; p.ranks = ranks;
   p.scalings = scalings; p.T = T; p.in = in; p.slots = slots; p.R = R; p.S = S;
-  p.nks = group_shrink_chunks(in);
-  static_assert(32 * kGsWarps == 512, "one chunk is 512 features");
+  p.chunk = group_shrink_chunk(in);
+  p.nks = ceil_div_i(in, p.chunk);
   *ksplit_out = p.nks;
-  p.off_red = round_up_i((slots + 1 + kGsWarps) * 4, 16);
   const int SR = S * R;
-  const size_t smem = (size_t)p.off_red + (size_t)kGsWarps * kStRows * SR * 4;
+  p.off_segs = round_up_i((slots + 1 + kGsWarps) * 4, 16);
+  p.off_red = round_up_i(p.off_segs + slots * 8, 16);
+  const size_t smem = (size_t)p.off_red + (size_t)kGsWarps * kStRows * (SR + 8) * 4;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3((unsigned)sms, 1, 1);

@@ -343,19 +343,22 @@ cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overl
                           const char** why);
 
 // Shrink over short segments (group_shrink.cu): row groups of 16, the input
-// features in chunks of 512 (at most 8), fp32 partial h per chunk; S*R in
-// {16, 32, 48, 64}.  Segments [seg_lo[s], seg_hi[s]), or CSR by slot
-// [seg_lo[s], seg_lo[s+1]) when seg_hi is null; A of pair slot_map[s] (s when
-// null).  *ksplit_out = the number of chunks.  allow_overlap: the
-// programmatic edge to the preceding kernel (x read and h written after it).
+// features in at most kGsMaxParts chunks of group_shrink_chunk(in) = 256 << k
+// features, fp32 partial h per chunk; S*R in {16, 32, 48, 64}, 8 <= in <=
+// kGsMaxIn.  Segments [seg_lo[s], seg_hi[s]), or CSR by slot [seg_lo[s],
+// seg_lo[s+1]) when seg_hi is null; A of pair slot_map[s] (s when null).
+// *ksplit_out = the number of chunks.  allow_overlap: the programmatic edge to
+// the preceding kernel (x read and h written after it).
+constexpr int kGsMaxIn = 4096;
+constexpr int kGsMaxParts = 8;
 bool group_shrink_supported(int S, int R, int in);
 cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const int* token_order,
                                 const int* seg_lo, const int* seg_hi, const int* slot_map,
                                 const int* ranks, const float* scalings, int T, int in,
                                 int slots, int R, int S, int* ksplit_out, cudaStream_t stream,
                                 bool allow_overlap);
-constexpr int kGsMaxIn = 4096;
-inline int group_shrink_chunks(int in) { return ceil_div_i(in, 512); }
+int group_shrink_chunk(int in);
+int group_shrink_chunks(int in);
 
 // The MoE fold grouped by (slot, expert) (moe_group.cu): per adapted expert,
 // its rows sorted by slot into token_order, group g = s * num_experts + e owning
@@ -368,9 +371,10 @@ cudaError_t moe_group_launch(const int* expert_offsets, const int* pair_index, c
                              uint32_t* flags, cudaStream_t stream);
 
 // Workspace bytes lora_apply_linear needs for these shapes in `regime` (AUTO
-// resolved with the real in_features), 0 if none (api.cu).
+// resolved with the real in_features, out and a workspace of ws_bytes), 0 if
+// none (api.cu).
 size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,
-                              int out);
+                              int out, size_t ws_bytes);
 
 // Launchers (bgmv.cu).  Return a cudaError_t from the launch.
 cudaError_t bgmv_launch(int mode, const BgmvParams& p, int max_items, cudaStream_t stream,

@@ -29,7 +29,7 @@
 namespace lora {
 void set_last_error(const char* msg);  // api.cu
 size_t apply_linear_workspace(int regime, int T, int in_features, int slots, int R, int S,
-                              int out);  // api.cu
+                              int out, size_t ws_bytes);  // api.cu
 }
 
 namespace {
@@ -57,7 +57,8 @@ lora_status lora_apply_linear_noalloc(const void* x, void* y, const void* a, con
   // them to (argument errors are left to lora_apply_linear to report)
   const size_t need =
       (out > 0 && out < (1LL << 30))
-          ? lora::apply_linear_workspace(regime, T, in_features, slots, R, num_slices, (int)out)
+          ? lora::apply_linear_workspace(regime, T, in_features, slots, R, num_slices, (int)out,
+                                         LORA_STATIC_SCRATCH_BYTES)
           : 0;
   if (need > (size_t)LORA_STATIC_SCRATCH_BYTES) {
     snprintf(msg, sizeof(msg),

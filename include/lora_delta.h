@@ -146,9 +146,11 @@ LORA_API lora_status lora_expand(void* y, const float* h, const void* b, const i
  *     workspace, then the streamed expand sums them (rows in 16-row groups,
  *     y by 16-byte loads and stores).  Takes num_slices*R in {16, 32, 48,
  *     64}, roundup(R, 16) <= 64 and in_features <= 4096 (else
- *     LORA_ERR_UNSUPPORTED).  AUTO takes it where it would take SGMV and
- *     T * in_features <= 2^22 with those shapes (lora_resolve_regime, which
- *     does not know in_features, answers SGMV there).
+ *     LORA_ERR_UNSUPPORTED).  AUTO takes it for those shapes with
+ *     512 <= T <= 8192, T * in_features <= 2^25 and T * out <= 2^26 when the
+ *     workspace given holds what STREAM needs, else it keeps its BGMV or
+ *     SGMV choice (lora_resolve_regime, which knows neither in_features nor
+ *     the workspace, answers with that choice).
  *   BGMV_SPLIT (only when asked for): one launch over every SM; the shrink is
  *     cut along the input features and the expand along the output columns
  *     into equal shares, and fp32 partial h pass through the workspace (each

@@ -162,19 +162,25 @@ def test_host_queries(lib):
     # per 512 input features, sized for in_features = 4096
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3,
                                   L.LORA_REGIME_STREAM) == 4096 + 8 * 256 * 3 * 16 * 4
-    # AUTO would stream T = 1024 with in_features up to 4096 (T * in <= 2^22):
-    # its workspace covers that as well as SGMV's four partial buffers
+    # AUTO streams 512 <= T <= 8192 with T * in_features <= 2^25 when the
+    # workspace holds it: lora_workspace_bytes covers eight partial buffers
+    # there (more than SGMV's four), nothing below T = 512, and SGMV's beyond
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 1024, 4, 16, 1) == \
         4096 + 8 * 1024 * 16 * 4
     assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 8192, 4, 16, 1) == \
-        4096 + 4 * 8192 * 16 * 4
+        4096 + 8 * 8192 * 16 * 4
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 512, 8, 16, 3) == \
+        4096 + 8 * 512 * 3 * 16 * 4
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 256, 32, 16, 3) == 0
+    assert L.lora_workspace_bytes(L.LORA_OP_APPLY_LINEAR, 16384, 4, 16, 1) == \
+        4096 + 4 * 16384 * 16 * 4
     # lora_resolve_regime does not know in_features: SGMV's shapes answer SGMV
     assert L.lora_resolve_regime(L.LORA_OP_APPLY_LINEAR, 2048, 4, 16, 1) == L.LORA_REGIME_SGMV
     # the grouped expert fold: token_order, the group tables (4096 groups x 4
-    # ints), then four fp32 partial h buffers; nothing for the per-chunk kernel
+    # ints), then eight fp32 partial h buffers; nothing for the per-chunk kernel
     rows, R, S = 16384, 16, 2
     assert L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, rows, 128, R, S) == \
-        rows * 4 + 4 * 4096 * 4 + 4 * rows * R * S * 4
+        rows * 4 + 4 * 4096 * 4 + 8 * rows * R * S * 4
     assert L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, rows, 128, R, S,
                                   L.LORA_REGIME_BGMV) == 0
     assert L.lora_workspace_bytes(L.LORA_OP_EXPERT_APPLY, rows, 128, 8, 1) == 0
