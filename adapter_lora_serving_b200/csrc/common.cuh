@@ -276,12 +276,12 @@ LORA_DEV int block_inclusive_scan(int v, int* scratch, int* total) {
 // is [slot_indptr[s], slot_indptr[s+1]), or [slot_indptr[s], seg_hi[s]) when
 // seg_hi is given (segments that need not abut, e.g. the MoE fold's
 // (slot, expert) groups).  seg_out (optional, shared memory): every slot's
-// (lo, hi) as read.
+// (lo, hi, rank, scaling bits) as read.
 template <int NT>
 LORA_DEV int plan_linear(const int* __restrict__ slot_indptr, const int* __restrict__ ranks,
                          const float* __restrict__ scalings, int slots, int T, int R, int tile,
                          int* prefix, int* scratch, uint32_t* flags, bool report,
-                         const int* __restrict__ seg_hi = nullptr, int2* seg_out = nullptr) {
+                         const int* __restrict__ seg_hi = nullptr, int4* seg_out = nullptr) {
   uint32_t bad = 0;
   int carry = 0;
   if (threadIdx.x == 0) prefix[0] = 0;
@@ -291,14 +291,16 @@ LORA_DEV int plan_linear(const int* __restrict__ slot_indptr, const int* __restr
     if (s < slots) {
       const int lo = slot_indptr[s];
       const int hi = seg_hi != nullptr ? seg_hi[s] : slot_indptr[s + 1];
-      if (seg_out != nullptr) seg_out[s] = make_int2(lo, hi);   // shared memory: the bounds as read
       const int r = ranks[s];
+      const float sc = scalings != nullptr ? scalings[s] : 1.0f;
+      // shared memory: the bounds, rank and scaling as read
+      if (seg_out != nullptr) seg_out[s] = make_int4(lo, hi, r, __float_as_int(sc));
       const bool seg_ok = lo >= 0 && lo <= hi && hi <= T;
       const bool rank_ok = r >= 0 && r <= R;
       if (!seg_ok) bad |= LORA_FLAG_BAD_INDPTR;
       if (!rank_ok) bad |= LORA_FLAG_BAD_RANK;
       bool take = seg_ok && rank_ok && r > 0;
-      if (take && scalings != nullptr && scalings[s] == 0.0f) take = false;
+      if (take && sc == 0.0f) take = false;
       if (take) cnt = (hi - lo + tile - 1) / tile;
     }
     int tot;

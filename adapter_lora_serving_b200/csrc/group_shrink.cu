@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
   extern __shared__ __align__(16) uint8_t smem[];
   int* prefix = reinterpret_cast<int*>(smem);                    // [slots + 1]
   int* scratch = prefix + p.slots + 1;                           // [kGsWarps]
-  int2* segs = reinterpret_cast<int2*>(smem + p.off_segs);       // [slots]
+  int4* segs = reinterpret_cast<int4*>(smem + p.off_segs);       // [slots]
   float* red = reinterpret_cast<float*>(smem + p.off_red);       // [kGsWarps][16][SRP]
   __shared__ int utok[kGsWarps][NSET][kStRows + 1];   // a unit's 16 row tokens and its chunk
   __shared__ int rtok[kGsWarps][kStRows];             // a team's 16 row tokens
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) group_shrink_kernel(const GShri
     const int g = (int)(u / p.nks);
     kc = (int)(u - (long long)g * p.nks);
     const int s = find_segment(prefix, p.slots, g);
-    const int2 sg = segs[s];
+    const int4 sg = segs[s];
     pair = p.slot_map != nullptr ? p.slot_map[s] : s;
     pa = sg.x + (g - prefix[s]) * kStRows + g8;
     hi = sg.y;
@@ -308,7 +308,7 @@ cudaError_t group_shrink_launch(const void* x, const void* a, float* h, const in
   *ksplit_out = p.nks;
   const int SR = S * R;
   p.off_segs = round_up_i((slots + 1 + kGsWarps) * 4, 16);
-  p.off_red = round_up_i(p.off_segs + slots * 8, 16);
+  p.off_red = round_up_i(p.off_segs + slots * 16, 16);
   const size_t smem = (size_t)p.off_red + (size_t)kGsWarps * kStRows * (SR + 8) * 4;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];

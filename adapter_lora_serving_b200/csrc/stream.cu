@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
   uint64_t* bfull = reinterpret_cast<uint64_t*>(smem);
   uint64_t* bempty = bfull + kStBBufs;
   int* prefix = reinterpret_cast<int*>(smem + p.off_prefix);
-  int2* segs = reinterpret_cast<int2*>(smem + p.off_segs);      // every slot's (lo, hi)
+  int4* segs = reinterpret_cast<int4*>(smem + p.off_segs);      // every slot's lo, hi, rank, scaling
   int* scratch = reinterpret_cast<int*>(smem + p.off_scratch);
   int* spec = reinterpret_cast<int*>(smem + p.off_spec);      // token_order read ahead
   int* ctok = reinterpret_cast<int*>(smem + p.off_ctok);      // tokens of the window
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int g = (int)(gw0 + e / kStRows);
       const int i = e % kStRows;
       const int s = find_segment(prefix, p.slots, g);
-      const int2 sg = segs[s];
+      const int4 sg = segs[s];
       const long long lo = sg.x;
       const long long hi = sg.y;
       const long long pos = lo + (long long)(g - prefix[s]) * kStRows + i;
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       }
       ctok[e] = tok;
       if (i == 0)
-        gmeta[e / kStRows] = make_int4(s, p.ranks[s], __float_as_int(p.scalings[s]), 0);
+        gmeta[e / kStRows] = make_int4(s, sg.z, sg.w, 0);
     }
     __syncthreads();
 
@@ -601,8 +601,8 @@ cudaError_t stream_launch(StreamParams& p, cudaStream_t stream, bool allow_overl
   int off = 2 * kStBBufs * 8;
   p.off_prefix = off;
   off += round_up_i((p.slots + 1) * 4, 16);
-  p.off_segs = off;
-  off += round_up_i(p.slots * 8, 16);
+  p.off_segs = round_up_i(off, 16);
+  off = p.off_segs + p.slots * 16;
   p.off_scratch = off;
   off += round_up_i(kStThreads / 32 * 4, 16);
   p.off_spec = off;
