@@ -575,21 +575,29 @@ def source_digest(kernel):
     return h.hexdigest()[:16]
 
 
+# The kernel with the largest share of each workload's step under AUTO (the
+# launch lists under profiles/).
+DOMINANT = {"tiny_linear": "bgmv_kernel", "decode_qkv": "bgmv_kernel",
+            "prefill_gate_up": "sgmv_expand_kernel", "embedding": "stream_kernel",
+            "moe_expert": "stream_kernel", "moe_router": "group_shrink_kernel"}
+
+
 def measured_traffic(name):
     """DRAM bytes per launch of the workload's dominant kernel from one ncu
-    capture (profiles/traffic.json), or None once that kernel's sources differ
-    from the ones the capture was taken at."""
+    capture (profiles/traffic.json), or None when there is none or that
+    kernel's sources differ from the ones the capture was taken at."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(name)
     except (OSError, ValueError):
-        return None, None
+        return None, DOMINANT.get(name)
     if not rec:
-        return None, None
+        return None, DOMINANT.get(name)
     kernel = rec.get("kernel")
-    if kernel not in KERNEL_SOURCES or rec.get("source_digest") != source_digest(kernel):
-        return None, kernel
+    if kernel != DOMINANT.get(name) or kernel not in KERNEL_SOURCES or \
+            rec.get("source_digest") != source_digest(kernel):
+        return None, DOMINANT.get(name)
     return rec.get("dram_bytes_per_launch"), kernel
 
 
@@ -675,7 +683,7 @@ def main():
                 "frac": round(step_gbs / hbm_peak, 4), "traffic": traffic,
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                 "algorithmic_bytes_per_step": int(wl.bytes),
-                "kernel": kname or "bgmv_kernel",
+                "kernel": kname,
                 "per_launch_us": round(kernel_s * 1e6, 3) if kernel_s else None}
 
     e2e = time_e2e(torch, wl, args.e2e_steps) if rank == 0 and not args.profile else None
