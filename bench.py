@@ -679,6 +679,9 @@ def main():
     kernel_s = sec / (args.steps * wl.launches_per_step) if wl.launches_per_step == 1 else None
     step_gbs = wl.bytes / (sec / args.steps) / 1e9
     traffic, kname = measured_traffic(name)
+    if args.regime != "auto":
+        # the captures behind traffic.json are of the AUTO regime's kernel
+        traffic, kname = None, None
     roofline = {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(step_gbs / hbm_peak, 4), "traffic": traffic,
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
