@@ -269,3 +269,16 @@ def test_unsupported_shapes_and_small_workspace():
                             err_flags=d.flags)
     assert e.value.status == "LORA_ERR_WORKSPACE"
     assert np.array_equal(host_bits(d.y), p.y)
+
+
+def test_no_live_slot_and_the_slot_limit():
+    """Every slot at rank 0 (or scaling 0): no row group, y bit-identical.  Then
+    LORA_MAX_SLOTS (4096) slots over 600 tokens: most slots empty, the plan's
+    tables at their largest in shared memory."""
+    p = W.random_linear(48, 300, 512, (64, 64), 5, 16, ranks=[0, 0, 0, 0, 0])
+    d = LinearDev(p)
+    _apply(d)
+    assert read_flags(d.flags) == 0
+    assert np.array_equal(host_bits(d.y), p.y)
+    q = W.random_linear(49, 600, 256, (128,), 4096, 16, dead_frac=0.05)
+    _check(q, "4096 slots")
