@@ -126,8 +126,8 @@ int resolve(int regime, int op, int T, int slots, int R, int S, int in_features 
 // Workspace bytes lora_apply_linear needs in regime `reg` (0: none).  SGMV:
 // the counter header (which it leaves alone), then the partial h buffers of
 // the split shrink.  BGMV_SPLIT: its counters and partials.  STREAM: the
-// counter header (which it leaves alone), then the partial h of every
-// 512-feature chunk.  BGMV: none.
+// counter header (which it leaves alone), then the partial h of every chunk
+// of the input features (at most eight).  BGMV: none.
 size_t apply_linear_need(int reg, int T, int in_features, int slots, int R, int S, int out) {
   if (T <= 0 || R <= 0 || S <= 0) return 0;
   if (reg == LORA_REGIME_SGMV) return lora::kWsCounterBytes + lora::sgmv_workspace_bytes(T, R, S);
@@ -604,8 +604,8 @@ lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* 
   if (workspace != nullptr && gneed > 0 && workspace_bytes >= gneed &&
       (long long)slots * num_experts <= lora::kMoeMaxGroups && in_features >= 64 &&
       lora::stream_supported(R)) {
-    // grouped fold: rows sorted by (slot, expert), then the SGMV shrink and
-    // expand over the groups' segments
+    // grouped fold: rows sorted by (slot, expert), then the short-segment
+    // (or SGMV) shrink and the streamed expand over the groups' segments
     if (!aligned16(workspace))
       return fail(LORA_ERR_INVALID, "%s: workspace is not 16-byte aligned", op);
     const int G = slots * num_experts;

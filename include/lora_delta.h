@@ -251,9 +251,11 @@ LORA_API lora_status lora_apply_embedding(const int32_t* ids, void* y, const voi
  * initialisation needed; 0 when the shapes are outside the SGMV rule R in
  * {16, 32, 64}, num_slices * R <= 128) and slots * num_experts <= 4096 and
  * in_features >= 64, it is grouped by (slot, expert): a device pass sorts
- * each adapted expert's rows by slot, then the tensor-core shrink and expand
- * tile every (slot, expert) group like a slot's tokens (three launches).
- * Otherwise the workspace is left unused.
+ * each adapted expert's rows by slot, then a shrink over 16-row groups
+ * (num_slices * R <= 64 and in_features <= 4096; else the tensor-core shrink)
+ * writes fp32 partial h into the workspace and the streamed expand folds it
+ * into every (slot, expert) group's rows (three launches).  Otherwise the
+ * workspace is left unused.
  */
 LORA_API lora_status lora_expert_apply(const void* x_sorted, void* y_sorted, const void* a,
                               const void* b, const int32_t* pair_index, const int32_t* ranks,
