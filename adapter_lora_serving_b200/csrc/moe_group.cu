@@ -47,16 +47,17 @@ struct MoeGroupParams {
 };
 
 // The row's group slot, or -1 when the row is left out (flags in *bad).
-// srank / sscal: the slots' ranks and scalings, read once into shared memory.
-LORA_DEV int classify_row(const MoeGroupParams& p, const int* srank, const float* sscal, int e,
-                          int rho, uint32_t* bad) {
+// srank / sscal / spair: the slots' ranks, scalings and pairs for expert e,
+// read once into shared memory.
+LORA_DEV int classify_row(const MoeGroupParams& p, const int* srank, const float* sscal,
+                          const int* spair, int rho, uint32_t* bad) {
   const int s = p.row_slot[rho];
   if (s == -1) return -1;
   if (s < -1 || s >= p.slots) {
     *bad |= LORA_FLAG_BAD_SLOT;
     return -1;
   }
-  const int pi = p.pair_index[(size_t)s * p.num_experts + e];
+  const int pi = spair[s];
   if (pi == -1) return -1;
   if (pi < -1 || pi >= p.num_pairs) {
     *bad |= LORA_FLAG_BAD_PAIR;
@@ -77,31 +78,31 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
   int* cur = sm + p.slots;     // [slots] next position per slot
   int* srank = cur + p.slots;  // [slots]
   float* sscal = reinterpret_cast<float*>(srank + p.slots);   // [slots]
-  int* cls = reinterpret_cast<int*>(sscal + p.slots);         // [kMgCache] row classes
+  int* spair = reinterpret_cast<int*>(sscal + p.slots);       // [slots] pair of (slot, e)
+  int* cls = spair + p.slots;                                 // [kMgCache] row classes
   __shared__ int scratch[kMgThreads / 32];
-  __shared__ int adapted;
   __shared__ int dead_cur;
   __shared__ uint32_t bad_all;
   const int e = blockIdx.x;
   const int E = p.num_experts;
   const int tid = threadIdx.x;
   if (tid == 0) {
-    adapted = 0;
     dead_cur = 0;
     bad_all = 0u;
   }
   // everything the classification needs besides the rows, in one round trip
   const int off0 = p.expert_offsets[e];
   const int off1 = p.expert_offsets[e + 1];
+  int mine = 0;   // this thread saw a pair for expert e
   for (int s = tid; s < p.slots; s += kMgThreads) {
     cnt[s] = 0;
     srank[s] = p.ranks[s];
     sscal[s] = p.scalings[s];
+    const int pi = p.pair_index[(size_t)s * E + e];
+    spair[s] = pi;
+    if (pi != -1) mine = 1;
   }
-  __syncthreads();
-  for (int s = tid; s < p.slots; s += kMgThreads)
-    if (p.pair_index[(size_t)s * E + e] != -1) adapted = 1;
-  __syncthreads();
+  const int adapted = __syncthreads_or(mine);
   int start = 0, end = 0;
   if (adapted) {
     start = off0;
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
   }
   uint32_t bad = 0;
   for (int rho = start + tid; rho < end; rho += kMgThreads) {
-    const int s = classify_row(p, srank, sscal, e, rho, &bad);
+    const int s = classify_row(p, srank, sscal, spair, rho, &bad);
     if (rho - start < kMgCache) cls[rho - start] = s;
     if (s >= 0) atomicAdd(&cnt[s], 1);
   }
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kMgThreads) moe_group_kernel(const MoeGroupPar
   for (int rho = start + tid; rho < end; rho += kMgThreads) {
     uint32_t unused = 0;
     const int s = rho - start < kMgCache ? cls[rho - start]
-                                         : classify_row(p, srank, sscal, e, rho, &unused);
+                                         : classify_row(p, srank, sscal, spair, rho, &unused);
     const int pos = s >= 0 ? atomicAdd(&cur[s], 1) : dead_lo + atomicAdd(&dead_cur, 1);
     p.token_order[pos] = rho;
   }
@@ -163,7 +164,7 @@ cudaError_t moe_group_launch(const int* expert_offsets, const int* pair_index, c
   p.seg_hi = seg_hi; p.g_rank = g_rank; p.g_scal = g_scal; p.flags = flags;
   p.rows_cap = rows_cap; p.num_experts = num_experts; p.slots = slots; p.num_pairs = num_pairs;
   p.R = R;
-  const size_t smem = (size_t)4 * slots * sizeof(int) + (size_t)kMgCache * sizeof(int);
+  const size_t smem = (size_t)5 * slots * sizeof(int) + (size_t)kMgCache * sizeof(int);
   if (smem > 48 * 1024) {
     const cudaError_t err = cudaFuncSetAttribute(
         moe_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
