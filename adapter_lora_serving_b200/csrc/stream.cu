@@ -272,10 +272,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
       }
     } else {
       // ---------------------------------------------------------- consumers
-      // units in order: block by block, the window's groups inside each block.
-      // y of unit u + D is requested while unit u is computed; the first D
-      // units' y goes out before h is read (a row that turns out to have no h
-      // -- an id outside the vocabulary -- is read and left alone).
+      // units in order: row group by row group, the blocks inside each group.
+      // y of unit u + D is requested while unit u is computed.
       uint4 ya[D], yb[D];
       int icb = cb0, igi = gi0, ireq = 0;  // next unit to request
       auto request = [&](uint4& ra, uint4& rb) {
@@ -285,8 +283,11 @@ __global__ void __launch_bounds__(kStThreads, 1)
         int sl, c0, ncols;
         block_cols(p, icb, sl, c0, ncols);
         if (cc < ncols) {
-          const int tA = ctok[igi * kStRows + g8];
-          const int tB = ctok[igi * kStRows + g8 + 8];
+          // a gathered h's rows are known once the ids are in (an id outside
+          // the vocabulary leaves its row alone: it is not read)
+          const int* rt = kH ? ctok : cval;
+          const int tA = rt[igi * kStRows + g8];
+          const int tB = rt[igi * kStRows + g8 + 8];
           if (tA >= 0) ra = *reinterpret_cast<const uint4*>(Y + ((size_t)tA * p.out + c0 + cc) * 2);
           if (tB >= 0) rb = *reinterpret_cast<const uint4*>(Y + ((size_t)tB * p.out + c0 + cc) * 2);
         }
@@ -295,8 +296,14 @@ __global__ void __launch_bounds__(kStThreads, 1)
           ++igi;
         }
       };
+      // a computed h (L2-resident partials) is summed while the first units'
+      // y is on its way; the ids and A columns of a gathered h go out first,
+      // ahead of the y stream in the DRAM queues, and y follows them (the
+      // two dependent loads took 3.8 us behind the y stream)
+      if (kH) {
 #pragma unroll
-      for (int j = 0; j < D; ++j) request(ya[j], yb[j]);
+        for (int j = 0; j < D; ++j) request(ya[j], yb[j]);
+      }
 
       const int ct = tid - 32;
       // h of the window's rows, every slice (zeros past the rank and for rows
@@ -375,6 +382,10 @@ __global__ void __launch_bounds__(kStThreads, 1)
         }
       }
       consumer_sync();
+      if (!kH) {
+#pragma unroll
+        for (int j = 0; j < D; ++j) request(ya[j], yb[j]);
+      }
 
       int pcb = cb0, pgi = gi0;            // unit being computed
       bool stop = false;
