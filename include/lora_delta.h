@@ -218,8 +218,10 @@ LORA_API lora_status lora_gather_shrink(const int32_t* ids, float* h, const void
  * expand; fused, h kept on chip).  A token whose id is outside [0, vocab)
  * contributes nothing and its row of y stays bit-identical.
  * Regimes: AUTO and STREAM run one launch over every SM that streams the y rows
- * of every live token through shared memory (roundup(R, 16) <= 64, else
- * AUTO takes one of the others); BGMV and SGMV run those regimes' kernels.
+ * of every live token in 16-row groups, 16-byte loads and stores in flight in
+ * registers (roundup(R, 16) <= 64, else AUTO takes one of the others); the
+ * rows of ids outside the vocabulary are not read.  BGMV and SGMV run those
+ * regimes' kernels.
  */
 LORA_API lora_status lora_apply_embedding(const int32_t* ids, void* y, const void* a, const void* b,
                                  const int32_t* ranks, const float* scalings,
