@@ -208,3 +208,20 @@ def test_split_regime_refuses_shapes_beyond_its_limits(lib):
     assert "BGMV_SPLIT" in lib.lora_last_error().decode()
     # within its limits but without a workspace: refused before launch
     assert _apply(lib, regime=L.LORA_REGIME_BGMV_SPLIT) == L.LORA_ERR_WORKSPACE
+
+
+def test_stream_regime_refuses_before_launch(lib):
+    S = L.LORA_REGIME_STREAM
+    ws = 1 << 20
+    # S*R outside {16, 32, 48, 64}, or in_features past 4096: unsupported
+    assert _apply(lib, R=32, out_slices=(32, 32, 32), regime=S, ws=ws, ws_bytes=1 << 30) == \
+        L.LORA_ERR_UNSUPPORTED
+    assert "STREAM" in lib.lora_last_error().decode()
+    assert _apply(lib, in_features=4104, regime=S, ws=ws, ws_bytes=1 << 30) == \
+        L.LORA_ERR_UNSUPPORTED
+    # the counter header and one chunk of partials are needed: one byte short
+    need = 4096 + 4 * 16 * 16
+    assert _apply(lib, regime=S, ws=ws, ws_bytes=need - 1) == L.LORA_ERR_WORKSPACE
+    assert _apply(lib, regime=S) == L.LORA_ERR_WORKSPACE
+    # a workspace that is not 16-byte aligned
+    assert _apply(lib, regime=S, ws=ws + 4, ws_bytes=need) == L.LORA_ERR_INVALID
